@@ -1,0 +1,75 @@
+"""Helpers shared by the GPU parity tests: moving generator arrays to the device, building
+states through the library's commit call, and the tolerance checks.
+
+Tolerances (block-hybrid decode step, one layer):
+  bf16 activations, fp32 states: max |gpu - oracle| <= 2e-2 and ||gpu - oracle|| / ||oracle|| <= 5e-3
+  fp32 activations and states:   ||gpu - oracle|| / ||oracle|| <= 1e-5 and
+                                 max |gpu - oracle| / max |oracle| <= 1e-5
+"""
+import numpy as np
+import torch
+
+from linear_attention_diffusion_hedgehog_b200 import bha
+
+TOL_BF16 = dict(max_abs=2e-2, rel_l2=5e-3)
+TOL_F32 = dict(rel_l2=1e-5, rel_max=1e-5)
+
+
+def dev(x, dtype):
+    return torch.from_numpy(np.ascontiguousarray(x)).to(device="cuda", dtype=dtype)
+
+
+def act_dtype(case):
+    return torch.bfloat16 if case.dtype == "bf16" else torch.float32
+
+
+def host64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def errors(got, want):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    diff = got - want
+    nref = np.linalg.norm(want)
+    return dict(
+        max_abs=float(np.abs(diff).max()) if diff.size else 0.0,
+        rel_l2=float(np.linalg.norm(diff) / nref) if nref > 0 else float(np.linalg.norm(diff)),
+        rel_max=float(np.abs(diff).max() / np.abs(want).max()) if diff.size and np.abs(want).max() > 0 else 0.0,
+    )
+
+
+def assert_close(got, want, tol, what=""):
+    e = errors(got, want)
+    assert np.isfinite(np.asarray(got)).all(), f"{what}: non-finite values"
+    for k, v in tol.items():
+        assert e[k] <= v, f"{what}: {k} = {e[k]:.3e} > {v:.1e} (all: {e})"
+    return e
+
+
+def build_states_on_gpu(case, block=32, dtype=None, num_slots=None):
+    """Fold every request's committed prefix into fresh zero states with the library's
+    commit call, `block` tokens at a time (prefix_lens must be multiples of `block`)."""
+    dtype = dtype or act_dtype(case)
+    R, Hkv, d, F = case.R, case.Hkv, case.d, case.F
+    slots = num_slots or R
+    S = torch.zeros((slots, Hkv, F, d), device="cuda", dtype=torch.float32)
+    Z = torch.zeros((slots, Hkv, F), device="cuda", dtype=torch.float32)
+    W = dev(case.W, dtype)
+    Kp = dev(case.K_pre, dtype)
+    Vp = dev(case.V_pre, dtype)
+    pl = case.prefix_lens
+    nblk = int((pl.max() + block - 1) // block) if R else 0
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for j in range(nblk):
+        lens = np.clip(pl - j * block, 0, block)
+        idx = np.concatenate([case.cu_pre[r] + j * block + np.arange(lens[r]) for r in range(R)]
+                             ).astype(np.int64)
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device="cuda")
+        ii = torch.from_numpy(idx).cuda()
+        Kb = Kp.index_select(0, ii).contiguous()
+        Vb = Vp.index_select(0, ii).contiguous()
+        bha.commit_block(cu, Kb, Vb, W, S, Z, max_block=block, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    return S, Z

@@ -1,0 +1,262 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on identical
+seeded inputs.  Tolerances are stated in tests/gpu_util.py."""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_diffusion_hedgehog_b200 import bha, inputs
+from oracle import bha_ref as ref
+from tests.gpu_util import (TOL_BF16, TOL_F32, act_dtype, assert_close, build_states_on_gpu,
+                            dev, host64)
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_states(case, reqs=None):
+    reqs = range(case.R) if reqs is None else reqs
+    S = np.zeros((case.R, case.Hkv, case.F, case.d))
+    Z = np.zeros((case.R, case.Hkv, case.F))
+    for r in reqs:
+        lo, hi = case.cu_pre[r], case.cu_pre[r + 1]
+        for g in range(case.Hkv):
+            S[r, g], Z[r, g] = ref.state_from_tokens(case.K_pre[lo:hi, g], case.V_pre[lo:hi, g],
+                                                     case.W[g])
+    return S, Z
+
+
+def run_hybrid(case, S, Z, alpha=None, state_slot=None, dtype=None):
+    dtype = dtype or act_dtype(case)
+    cu = torch.tensor(case.cu_blk, dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O = bha.hybrid_attn(cu, dev(case.Q, dtype), dev(case.K, dtype), dev(case.V, dtype), S, Z,
+                        dev(case.W, dtype), max_block=int(max(case.block_lens.max(), 1)),
+                        alpha=None if alpha is None else dev(alpha, torch.float32),
+                        state_slot=state_slot, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    return O
+
+
+def rows_of(case, reqs):
+    return np.concatenate([np.arange(case.cu_blk[r], case.cu_blk[r + 1]) for r in reqs])
+
+
+# ------------------------------------------------------------------- tiny fp32 case
+
+@pytest.mark.parametrize("with_alpha", [False, True])
+def test_tiny_fp32_decode_step_and_commit(with_alpha):
+    c = inputs.tiny_case(seed=0, with_alpha=with_alpha)
+    S, Z = build_states_on_gpu(c, block=8)
+    So, Zo = oracle_states(c)
+    assert_close(host64(S), So, TOL_F32, "S after 3 commits")
+    assert_close(host64(Z), Zo, TOL_F32, "Z after 3 commits")
+    O = run_hybrid(c, S, Z, alpha=c.alpha)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, So, Zo, c.W, c.alpha)
+    assert_close(host64(O), want, TOL_F32, "O")
+
+
+# ------------------------------------------------------------------- feature map
+
+@pytest.mark.parametrize("dt,out_dt", [("bf16", torch.float32), ("bf16", torch.bfloat16),
+                                       ("f32", torch.float32)])
+def test_featuremap(dt, out_dt):
+    c = inputs.decode_case(R=3, Hq=8, Hkv=2, d=128, F=256, block_lens=[32, 7, 1], prefix_lens=0,
+                           seed=21, dtype=dt)
+    x = dev(c.Q, act_dtype(c))
+    phi = bha.featuremap(x, dev(c.W, act_dtype(c)), out_dtype=out_dt)
+    torch.cuda.synchronize()
+    want = ref.featuremap(c.Q, c.W)
+    got = host64(phi)
+    if out_dt == torch.float32 and dt == "f32":
+        assert_close(got, want, TOL_F32, "phi")
+    elif out_dt == torch.float32:
+        assert_close(got, want, dict(rel_l2=1e-5, max_abs=1e-6), "phi")
+    else:  # bf16 output: one rounding of values in (0, 1)
+        assert_close(got, want, dict(rel_l2=5e-3, max_abs=4e-3), "phi")
+    # each half of phi sums to 1
+    np.testing.assert_allclose(got[..., :128].sum(-1), 1.0, atol=2e-2 if out_dt == torch.bfloat16 else 1e-5)
+
+
+def test_featuremap_odd_dims_and_head_map():
+    c = inputs.decode_case(R=2, Hq=6, Hkv=3, d=40, F=70, block_lens=[5, 9], prefix_lens=0, seed=5,
+                           dtype="f32")
+    phi = bha.featuremap(dev(c.Q, torch.float32), dev(c.W, torch.float32))
+    torch.cuda.synchronize()
+    assert_close(host64(phi), ref.featuremap(c.Q, c.W), TOL_F32, "phi")
+
+
+# ------------------------------------------------------------------- decode step, bf16
+
+def test_decode_step_one_layer_128_requests():
+    """128 requests, 16 query / 4 KV heads, d 128, F 256, 32-token blocks, 1024-token prefixes
+    folded into S/Z by 32 commits; every output row of 8 sampled requests checked."""
+    c = inputs.decode_case(R=128, Hq=16, Hkv=4, d=128, F=256, block_lens=32, prefix_lens=1024,
+                           seed=2, dtype="bf16")
+    S, Z = build_states_on_gpu(c, block=32)
+    O = run_hybrid(c, S, Z)
+    reqs = np.random.default_rng(0).choice(128, 8, replace=False)
+    So, Zo = oracle_states(c, reqs)
+    for r in reqs:
+        assert_close(host64(S[r]), So[r], TOL_BF16, f"S[{r}]")
+        assert_close(host64(Z[r]), Zo[r], TOL_BF16, f"Z[{r}]")
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, So, Zo, c.W)
+    rows = rows_of(c, reqs)
+    assert_close(host64(O)[rows], want[rows], TOL_BF16, "O")
+
+
+def test_decode_step_ragged_slots_gate_isolated_states():
+    """Ragged blocks (0, 1, 31, 32 tokens), a permuted slot map, the sigmoid gate, and
+    directly drawn states, so the cross-block read is checked on its own."""
+    lens = [32, 0, 1, 31, 17, 32, 8, 2]
+    c = inputs.decode_case(R=8, Hq=16, Hkv=4, d=128, F=256, block_lens=lens, prefix_lens=0,
+                           seed=33, dtype="bf16", with_alpha=True)
+    S_np, Z_np = inputs.random_states(10, 4, 256, 128, prefix_len=700, seed=8)
+    slots = np.array([3, 9, 0, 5, 1, 2, 8, 6], dtype=np.int32)
+    S, Z = dev(S_np, torch.float32), dev(Z_np, torch.float32)
+    O = run_hybrid(c, S, Z, alpha=c.alpha, state_slot=torch.tensor(slots, device="cuda"))
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, S_np, Z_np, c.W, c.alpha, slots)
+    assert_close(host64(O), want, TOL_BF16, "O")
+
+
+def test_empty_prefix_is_block_softmax():
+    c = inputs.decode_case(R=4, Hq=16, Hkv=4, d=128, F=256, block_lens=[32, 5, 32, 1],
+                           prefix_lens=0, seed=4, dtype="bf16", with_alpha=True)
+    S = torch.zeros((4, 4, 256, 128), device="cuda")
+    Z = torch.zeros((4, 4, 256), device="cuda")
+    O = run_hybrid(c, S, Z, alpha=c.alpha)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, np.zeros((4, 4, 256, 128)),
+                           np.zeros((4, 4, 256)), c.W, c.alpha)
+    assert_close(host64(O), want, TOL_BF16, "O")
+
+
+def test_permuting_block_tokens_permutes_outputs():
+    c = inputs.decode_case(R=2, Hq=16, Hkv=4, d=128, F=256, block_lens=32, prefix_lens=0,
+                           seed=12, dtype="bf16")
+    S_np, Z_np = inputs.random_states(2, 4, 256, 128, prefix_len=300, seed=1)
+    S, Z = dev(S_np, torch.float32), dev(Z_np, torch.float32)
+    O = host64(run_hybrid(c, S, Z))
+    perm = np.concatenate([np.random.default_rng(3).permutation(32), 32 + np.arange(32)])
+    c.Q, c.K, c.V = c.Q[perm], c.K[perm], c.V[perm]
+    Op = host64(run_hybrid(c, S, Z))
+    assert_close(Op, O[perm], dict(max_abs=2e-2, rel_l2=1e-3), "permuted")
+
+
+# ------------------------------------------------------------------- commit, bf16
+
+def test_commit_one_block_onto_31_and_32_sequential():
+    """Fold a 32-token block into states holding 31 earlier blocks (128 requests x 4 KV
+    heads) and compare with a one-shot build over all 32 blocks."""
+    c = inputs.decode_case(R=128, Hq=4, Hkv=4, d=128, F=256, block_lens=32, prefix_lens=32 * 32,
+                           seed=3, dtype="bf16")
+    S, Z = build_states_on_gpu(c, block=32)   # 32 sequential commits from zero
+    reqs = np.random.default_rng(1).choice(128, 6, replace=False)
+    So, Zo = oracle_states(c, reqs)
+    for r in reqs:
+        assert_close(host64(S[r]), So[r], TOL_BF16, f"S[{r}] after 32 commits")
+        assert_close(host64(Z[r]), Zo[r], TOL_BF16, f"Z[{r}] after 32 commits")
+    # 31 blocks then the last one as a separate commit of the active block rows
+    c31 = inputs.decode_case(R=128, Hq=4, Hkv=4, d=128, F=256, block_lens=32, prefix_lens=31 * 32,
+                             seed=3, dtype="bf16")
+    S31, Z31 = build_states_on_gpu(c31, block=32)
+    cu = torch.tensor(c31.cu_blk, dtype=torch.int32, device="cuda")
+    bha.commit_block(cu, dev(c31.K, torch.bfloat16), dev(c31.V, torch.bfloat16),
+                     dev(c31.W, torch.bfloat16), S31, Z31, max_block=32)
+    torch.cuda.synchronize()
+    for r in reqs:
+        lo, hi = c31.cu_pre[r], c31.cu_pre[r + 1]
+        for g in range(4):
+            Kall = np.concatenate([c31.K_pre[lo:hi, g], c31.K[32 * r:32 * r + 32, g]])
+            Vall = np.concatenate([c31.V_pre[lo:hi, g], c31.V[32 * r:32 * r + 32, g]])
+            So1, Zo1 = ref.state_from_tokens(Kall, Vall, c31.W[g])
+            assert_close(host64(S31[r, g]), So1, TOL_BF16, f"S[{r},{g}] 31+1")
+            assert_close(host64(Z31[r, g]), Zo1, TOL_BF16, f"Z[{r},{g}] 31+1")
+
+
+def test_commit_ragged_with_slots_and_empty_blocks():
+    lens = [0, 5, 32, 1, 17]
+    c = inputs.decode_case(R=5, Hq=4, Hkv=4, d=128, F=256, block_lens=lens, prefix_lens=0, seed=6,
+                           dtype="bf16")
+    S_np, Z_np = inputs.random_states(7, 4, 256, 128, prefix_len=64, seed=2)
+    slots = np.array([6, 0, 3, 2, 5], dtype=np.int32)
+    S, Z = dev(S_np, torch.float32), dev(Z_np, torch.float32)
+    cu = torch.tensor(c.cu_blk, dtype=torch.int32, device="cuda")
+    bha.commit_block(cu, dev(c.K, torch.bfloat16), dev(c.V, torch.bfloat16),
+                     dev(c.W, torch.bfloat16), S, Z, max_block=32,
+                     state_slot=torch.tensor(slots, device="cuda"))
+    torch.cuda.synchronize()
+    So, Zo = ref.commit_block(c.cu_blk, c.K, c.V, c.W, S_np, Z_np, slots)
+    assert_close(host64(S), So, TOL_BF16, "S")
+    assert_close(host64(Z), Zo, TOL_BF16, "Z")
+    np.testing.assert_array_equal(host64(S[6]), S_np[6])   # b = 0: untouched
+    np.testing.assert_array_equal(host64(S[1]), S_np[1])   # no request: untouched
+
+
+# ------------------------------------------------------------------- generic dims
+
+def test_generic_max_dims_fp32():
+    """Largest dims the library accepts: d 256, F 512, a 128-token block (fp32)."""
+    c = inputs.decode_case(R=2, Hq=2, Hkv=1, d=256, F=512, block_lens=[128, 3], prefix_lens=[128, 0],
+                           seed=13, dtype="f32", with_alpha=True)
+    S, Z = build_states_on_gpu(c, block=128)
+    So, Zo = oracle_states(c)
+    assert_close(host64(S), So, TOL_F32, "S")
+    O = run_hybrid(c, S, Z, alpha=c.alpha)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, So, Zo, c.W, c.alpha)
+    assert_close(host64(O), want, TOL_F32, "O")
+
+
+def test_small_odd_dims_bf16():
+    c = inputs.decode_case(R=3, Hq=6, Hkv=2, d=24, F=20, block_lens=[7, 1, 13], prefix_lens=[9, 0, 30],
+                           seed=17, dtype="bf16")
+    S, Z = build_states_on_gpu(c, block=16)
+    So, Zo = oracle_states(c)
+    O = run_hybrid(c, S, Z)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, So, Zo, c.W)
+    assert_close(host64(O), want, TOL_BF16, "O")
+
+
+# ------------------------------------------------------------------- device-side validation
+
+def test_bad_cu_blk_sets_dev_err_and_skips():
+    c = inputs.decode_case(R=2, Hq=4, Hkv=4, d=128, F=256, block_lens=[16, 16], prefix_lens=0,
+                           seed=1, dtype="bf16")
+    S = torch.zeros((2, 4, 256, 128), device="cuda")
+    Z = torch.zeros((2, 4, 256), device="cuda")
+    cu = torch.tensor([0, 20, 32], dtype=torch.int32, device="cuda")   # block 0 longer than 16
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O = torch.full((32, 4, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    bha.hybrid_attn(cu, dev(c.Q, torch.bfloat16), dev(c.K, torch.bfloat16),
+                    dev(c.V, torch.bfloat16), S, Z, dev(c.W, torch.bfloat16), max_block=16,
+                    out=O, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == bha.BHA_ERR_INVALID
+    assert torch.all(O[:20] == 7.0)           # request 0 skipped
+    assert not torch.all(O[20:] == 7.0)       # request 1 computed
+    bad_slot = torch.tensor([0, 5], dtype=torch.int32, device="cuda")
+    err.zero_()
+    bha.commit_block(torch.tensor([0, 16, 32], dtype=torch.int32, device="cuda"),
+                     dev(c.K, torch.bfloat16), dev(c.V, torch.bfloat16), dev(c.W, torch.bfloat16),
+                     S, Z, max_block=16, state_slot=bad_slot, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == bha.BHA_ERR_INVALID
+
+
+# ------------------------------------------------------------------- softmax teacher
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_full_prefix_teacher(dt):
+    R, Hq, Hkv, d, cap = 3, 8, 2, 128, 300
+    kv_len = np.array([300, 33, 0], dtype=np.int32)
+    lens = np.array([32, 1, 4])
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    rng = np.random.default_rng(5)
+    cast = inputs.bf16_round if dt == "bf16" else (lambda x: x.astype(np.float32))
+    Q = cast(rng.standard_normal((cu[-1], Hq, d)).astype(np.float32))
+    Kc = cast(rng.standard_normal((R, Hkv, cap, d)).astype(np.float32))
+    Vc = cast(rng.standard_normal((R, Hkv, cap, d)).astype(np.float32))
+    tdt = torch.bfloat16 if dt == "bf16" else torch.float32
+    O = bha.full_prefix_attn(torch.tensor(cu, device="cuda"), torch.tensor(kv_len, device="cuda"),
+                             dev(Q, tdt), dev(Kc, tdt), dev(Vc, tdt), max_block=32)
+    torch.cuda.synchronize()
+    want = ref.full_prefix_attn(cu, kv_len, Q, Kc, Vc)
+    assert_close(host64(O), want, TOL_BF16 if dt == "bf16" else TOL_F32, "O")
