@@ -56,6 +56,19 @@ int bha_kernel_variant(const bha_dims* dims, int32_t which) {
   const int s = check_dims(dims);
   if (s != BHA_OK) return s;
   if (which < 0 || which > 3) return BHA_ERR_INVALID;
+  const bool bf16 = dims->act_dtype == BHA_BF16;
+  if (which == 1) {
+    bha::HybridArgs a{};
+    a.R = dims->num_requests;
+    a.Hq = dims->num_q_heads;
+    a.Hkv = dims->num_kv_heads;
+    a.d = dims->head_dim;
+    a.F = dims->feature_dim;
+    a.Bmax = dims->max_block;
+    a.T = dims->total_tokens;
+    a.num_slots = dims->num_slots;
+    return bha::hybrid_tc_supports(a, bf16) ? 1 : 0;
+  }
   return 0;
 }
 
@@ -94,8 +107,10 @@ int bha_hybrid_attn(const bha_dims* dims, const int32_t* cu_blk, const int32_t* 
   bha::HybridArgs a{cu_blk, state_slot, Q, K, V, S, Z, W, alpha, O, dev_err,
                     dims->num_requests, dims->num_q_heads, dims->num_kv_heads, dims->head_dim,
                     dims->feature_dim, dims->max_block, dims->total_tokens, dims->num_slots};
-  return launch_status(
-      bha::launch_hybrid_simt(a, dims->act_dtype == BHA_BF16, static_cast<cudaStream_t>(stream)));
+  const bool bf16 = dims->act_dtype == BHA_BF16;
+  if (bha::hybrid_tc_supports(a, bf16))
+    return launch_status(bha::launch_hybrid_tc(a, static_cast<cudaStream_t>(stream)));
+  return launch_status(bha::launch_hybrid_simt(a, bf16, static_cast<cudaStream_t>(stream)));
 }
 
 int bha_commit_block(const bha_dims* dims, const int32_t* cu_blk, const int32_t* state_slot,

@@ -1,6 +1,8 @@
 // Internal kernel-argument structs and launcher declarations (not part of the C ABI).
 #pragma once
 
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -46,6 +48,29 @@ struct FullPrefixArgs {
   int64_t kv_capacity;
   int R, Hq, Hkv, d, Bmax, T;
 };
+
+// Parameters of the tensor-core decode-step kernel (hybrid_tc.cu); the tensor maps describe
+// Q, K, V, W and S for the Tensor Memory Accelerator.
+struct TcHybridParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_w, tm_s;
+  const int32_t* cu_blk;
+  const int32_t* state_slot;
+  const float* Z;
+  const float* alpha;
+  __nv_bfloat16* O;
+  int32_t* dev_err;
+  int R, Hq, Hkv, T, Bmax, num_slots;
+  long long wait_limit;  // SM cycles a bounded wait may spin before giving up
+};
+
+// host helpers shared by the tensor-core launchers (hybrid_tc.cu)
+bool make_tensor_map(CUtensorMap* m, bool f32, int rank, const void* base, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box, bool swizzle_atom32);
+int device_sm_count();
+
+// tensor-core kernels
+bool hybrid_tc_supports(const HybridArgs& a, bool act_bf16);
+cudaError_t launch_hybrid_tc(const HybridArgs& a, cudaStream_t st);
 
 // generic CUDA-core kernels (simt.cu)
 bool simt_supports(int d, int F, int Bmax);

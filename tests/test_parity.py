@@ -260,3 +260,47 @@ def test_full_prefix_teacher(dt):
     torch.cuda.synchronize()
     want = ref.full_prefix_attn(cu, kv_len, Q, Kc, Vc)
     assert_close(host64(O), want, TOL_BF16 if dt == "bf16" else TOL_F32, "O")
+
+
+def test_tensor_core_path_is_taken_for_the_serving_shape():
+    d = bha.make_dims(128, 16, 4, 128, 256, 32, 4096, 128, torch.bfloat16)
+    assert bha.kernel_variant(d, 1) == 1
+    d32 = bha.make_dims(128, 16, 4, 128, 256, 32, 4096, 128, torch.float32)
+    assert bha.kernel_variant(d32, 1) == 0   # fp32 activations take the fp32 CUDA-core path
+
+
+def test_linear_branch_dominant_states():
+    """Large S and small Z make phi(q)^T S carry most of the output, so the feature map and
+    the state contraction are checked directly (not hidden behind the softmax branch)."""
+    c = inputs.decode_case(R=16, Hq=16, Hkv=4, d=128, F=256, block_lens=32, prefix_lens=0, seed=44,
+                           dtype="bf16")
+    rng = np.random.default_rng(9)
+    S_np = (5.0 * rng.standard_normal((16, 4, 256, 128))).astype(np.float32)
+    Z_np = rng.uniform(0.0, 0.5, size=(16, 4, 256)).astype(np.float32)
+    O = run_hybrid(c, dev(S_np, torch.float32), dev(Z_np, torch.float32))
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, S_np, Z_np, c.W)
+    assert_close(host64(O), want, TOL_BF16, "O")
+
+
+def test_zero_weight_closed_form_full_size():
+    """W = 0 makes phi uniform (1/128), so with states built from P prefix tokens
+    out_i = (sum_j a_ij v_j + (2/128) sum_t v_t) / (sum_j a_ij + 2P/128); checked at the serving
+    size (128 requests, 1024-token prefixes) without the oracle."""
+    c = inputs.decode_case(R=128, Hq=16, Hkv=4, d=128, F=256, block_lens=32, prefix_lens=1024,
+                           seed=5, dtype="bf16")
+    c.W = np.zeros_like(c.W)
+    S, Z = build_states_on_gpu(c, block=32)
+    O = host64(run_hybrid(c, S, Z))
+    P, Fh, G = 1024, 128, 4
+    Vsum = c.V_pre.astype(np.float64).reshape(128, P, 4, 128).sum(axis=1)          # [R, Hkv, d]
+    q = c.Q.astype(np.float64).reshape(128, 32, 16, 128)
+    k = c.K.astype(np.float64).reshape(128, 32, 4, 128)
+    v = c.V.astype(np.float64).reshape(128, 32, 4, 128)
+    kh = np.repeat(k, G, axis=2)
+    vh = np.repeat(v, G, axis=2)
+    s = np.einsum("rihd,rjhd->rhij", q, kh) / np.sqrt(128.0)
+    a = np.exp(s)
+    num = np.einsum("rhij,rjhd->rihd", a, vh) + (2.0 / Fh) * np.repeat(Vsum, G, axis=1)[:, None]
+    den = a.sum(-1).transpose(0, 2, 1)[..., None] + 2.0 * P / Fh
+    want = (num / den).reshape(4096, 16, 128)
+    assert_close(O, want, TOL_BF16, "O (closed form)")
