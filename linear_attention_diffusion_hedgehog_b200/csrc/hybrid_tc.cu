@@ -12,20 +12,22 @@
 // once per unit.  A persistent grid walks the units; unit u is (r = u / Hkv, g = u % Hkv),
 // so a CTA whose grid stride is a multiple of Hkv keeps one W_g resident.
 //
-// Roles (192 threads):
-//   warp 0     TMA producer: Q/K/V/Z of the next unit into a double buffer, W_g when g
-//              changes, and S_g in 32-row fp32 chunks through a 4-stage ring.
+// Roles (320 threads):
+//   warp 0     TMA producer.  Q/K (single buffer, refilled once the unit's score MMA has
+//              read them), V/Z (refilled after the unit's P.V MMA), W_g when g changes, and
+//              S_g as eight 32-row fp32 chunks, one ring stage each, so a whole unit's state
+//              streams in while the previous unit is still being contracted.
 //   warp 1     TMEM owner and MMA issuer (one thread):
-//                u   = Q W_g                 bf16 x bf16 -> fp32  TMEM cols [0, 128)
-//                s   = Q K_g^T               bf16 x bf16 -> fp32  TMEM cols [256, 288)
-//                acc = P V_g                 bf16 x bf16 -> fp32  TMEM cols [384, 512)
-//                acc += phi' S_g             tf32 (A from TMEM) x tf32 (S straight from the
-//                                            TMA-loaded fp32 tile)
-//   warps 2-5  one thread per tile row: block softmax (row max m over the block, P =
-//              w e^{s/sqrt d - m} in bf16), the feature map phi' = e^{-m} [softmax(u),
-//              softmax(-u)] written back over u in TMEM (cols [0, 256)), the linear
-//              denominator e^{-m} phi.Z on CUDA cores, then the epilogue
-//              out = acc / (w sum_j P + e^{-m} phi.Z) stored as bf16.
+//                u   = Q W_g          bf16 x bf16 -> fp32   TMEM cols [256, 384)
+//                s   = Q K_g^T        bf16 x bf16 -> fp32   TMEM cols [384, 416)
+//                acc = P V_g          bf16 x bf16 -> fp32   TMEM cols [384, 512) (after s is read)
+//                acc += phi' S_g      tf32, A = phi' from TMEM cols [0, 256), B = the fp32 S
+//                                     tile exactly as TMA delivered it
+//   warps 2-9  two threads per tile row (warps 2-5: softmax(u) half, warps 6-9: softmax(-u)
+//              half): block softmax (row max m over the block's keys, P = w e^{s/sqrt d - m}
+//              in bf16), that thread's half of phi' = e^{-m} [softmax(u), softmax(-u)] into
+//              TMEM, its half of the linear denominator e^{-m} phi.Z on CUDA cores, then the
+//              epilogue out = acc / (w sum_j P + e^{-m} phi.Z) for 64 of the 128 columns.
 // The shift m cancels between numerator and denominator; folding e^{-m} into phi and w
 // into P lets both branches share one TMEM accumulator.
 //
@@ -46,22 +48,23 @@ constexpr int kFh = 128;
 constexpr int kG = 4;
 constexpr int kBlk = 32;
 constexpr int kM = kG * kBlk;  // 128 tile rows
-constexpr int kStages = 4;
+constexpr int kStages = 8;  // a whole unit of S in flight
 constexpr int kChunk = 32;  // F rows of S per stage
 constexpr int kChunks = kF / kChunk;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA issuer, 8 softmax / epilogue warps
 
 constexpr uint32_t kQBytes = kM * kD * 2;      // 32 KiB
 constexpr uint32_t kKBytes = kBlk * kD * 2;    // 8 KiB
 constexpr uint32_t kZBytes = kF * 4;           // 1 KiB
 constexpr uint32_t kWBytes = kD * kFh * 2;     // 32 KiB
 constexpr uint32_t kSBytes = kChunk * kD * 4;  // 16 KiB
-constexpr uint32_t kPBytes = kM * 128;         // 16 KiB (128-byte rows, 64 used)
+constexpr uint32_t kPBytes = kM * 64;          // 8 KiB (64-byte rows, 64-byte swizzle)
 
 // TMEM columns
-constexpr uint32_t kColU = 0;     // u, then phi' (256 columns)
-constexpr uint32_t kColS = 256;   // block scores (32 columns)
-constexpr uint32_t kColAcc = 384; // output accumulator (128 columns)
+constexpr uint32_t kColPhi = 0;    // phi' (256 columns): A operand of the state read
+constexpr uint32_t kColS = 224;    // block scores (32 columns), read before phi' overwrites them
+constexpr uint32_t kColU = 256;    // u = Q W_g (128 columns)
+constexpr uint32_t kColAcc = 384;  // output accumulator (128 columns)
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kIdQW = tc::instr_desc(1, 0, 1, kM, kFh);
@@ -70,14 +73,15 @@ constexpr uint32_t kIdPV = tc::instr_desc(1, 0, 1, kM, kD);
 constexpr uint32_t kIdPS = tc::instr_desc(2, 0, 1, kM, kD);
 
 struct __align__(1024) Smem {
-  uint8_t q[2][kQBytes];      // [d half][128 rows][128 B], 128-byte swizzle
+  uint8_t q[kQBytes];         // [d half][128 rows][128 B], 128-byte swizzle
   uint8_t w[kWBytes];         // [f half][128 rows of d][128 B]
-  uint8_t s[kStages][kSBytes];// [d quarter][32 rows of f][128 B]
-  uint8_t k[2][kKBytes];      // [d half][32 rows][128 B]
-  uint8_t v[2][kKBytes];
-  uint8_t p[kPBytes];         // [128 rows][128 B], first 64 B of each row used
-  float z[2][kF];
-  uint64_t qkv_full[2], qkv_empty[2], s_full[kStages], s_empty[kStages];
+  uint8_t s[kStages][kSBytes];// [d quarter][32 rows of f][128 B], 128-byte swizzle, 32-byte atoms
+  uint8_t k[kKBytes];         // [d half][32 rows][128 B]
+  uint8_t v[kKBytes];
+  uint8_t p[kPBytes];         // [128 rows][64 B], 64-byte swizzle
+  float z[kF];
+  float red[2][kM];           // per-row linear-denominator halves
+  uint64_t qk_full, qk_empty, vz_full, vz_empty, s_full[kStages], s_empty[kStages];
   uint64_t w_full, u_full, phi_ready, acc_full, acc_empty, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -117,19 +121,19 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
   const int units = p.R * p.Hkv;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&sm.qkv_full[i], 1);
-      tc::mbar_init(&sm.qkv_empty[i], 1);
-    }
+    tc::mbar_init(&sm.qk_full, 1);
+    tc::mbar_init(&sm.qk_empty, 1);
+    tc::mbar_init(&sm.vz_full, 1);
+    tc::mbar_init(&sm.vz_empty, 1);
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&sm.s_full[i], 1);
       tc::mbar_init(&sm.s_empty[i], 1);
     }
     tc::mbar_init(&sm.w_full, 1);
     tc::mbar_init(&sm.u_full, 1);
-    tc::mbar_init(&sm.phi_ready, 4);
+    tc::mbar_init(&sm.phi_ready, 8);
     tc::mbar_init(&sm.acc_full, 1);
-    tc::mbar_init(&sm.acc_empty, 4);
+    tc::mbar_init(&sm.acc_empty, 8);
     tc::mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     tc::fence_barrier_init();
@@ -152,115 +156,93 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // Each buffer is refilled as soon as its last reader is done: Q/K after the unit's
+    // score MMA, V/Z after its P.V MMA, S stage c after the state-read MMAs of chunk c.
+    // With one stage per S chunk, unit k+1's whole state streams in while unit k's MMAs run.
     if (lane == 0) {
-      int k = 0, q = 0, g_res = -1;
+      int k = 0, g_res = -1;
       uint32_t w_loads = 0;
-      int armed_qkv[2] = {-1, -1};  // phase last armed per buffer (for the final drain)
-      int armed_s[kStages] = {-1, -1, -1, -1};
-      int armed_w = -1;
+      int armed_qk = -1, armed_vz = -1, armed_w = -1;
+      int armed_s[kStages];
+#pragma unroll
+      for (int i = 0; i < kStages; ++i) armed_s[i] = -1;
       bool ok = true;
-      Unit cur, nxt;
-      int u = blockIdx.x;
-      bool have = false;
-      for (; u < units; u += gridDim.x)
-        if (decode_unit(p, u, true, &cur)) { have = true; break; }
-
-      auto issue_w = [&](int g) {
-        tc::mbar_arrive_expect_tx(&sm.w_full, kWBytes);
-        tc::tma_load_2d(sm.w, &p.tm_w, &sm.w_full, 0, g * kD);
-        tc::tma_load_2d(sm.w + kWBytes / 2, &p.tm_w, &sm.w_full, 64, g * kD);
-        armed_w = w_loads & 1;
-        ++w_loads;
-      };
-      auto issue_qkv = [&](int kk, const Unit& x) -> bool {
-        const int buf = kk & 1, j = kk >> 1;
-        if (j >= 1 && !tc::mbar_wait(&sm.qkv_empty[buf], (j - 1) & 1, abort_flag, lim)) return false;
-        tc::mbar_arrive_expect_tx(&sm.qkv_full[buf], kQBytes + 2 * kKBytes + kZBytes);
-        uint64_t* bar = &sm.qkv_full[buf];
-        tc::tma_load_3d(sm.q[buf], &p.tm_q, bar, 0, kG * x.g, x.lo);
-        tc::tma_load_3d(sm.q[buf] + kQBytes / 2, &p.tm_q, bar, 64, kG * x.g, x.lo);
-        tc::tma_load_3d(sm.k[buf], &p.tm_k, bar, 0, x.g, x.lo);
-        tc::tma_load_3d(sm.k[buf] + kKBytes / 2, &p.tm_k, bar, 64, x.g, x.lo);
-        tc::tma_load_3d(sm.v[buf], &p.tm_v, bar, 0, x.g, x.lo);
-        tc::tma_load_3d(sm.v[buf] + kKBytes / 2, &p.tm_v, bar, 64, x.g, x.lo);
-        tc::bulk_load(sm.z[buf], p.Z + ((size_t)x.slot * p.Hkv + x.g) * kF, kZBytes, bar);
-        armed_qkv[buf] = j & 1;
-        return true;
-      };
-
-      if (have) {
-        issue_w(cur.g);
-        g_res = cur.g;
-        ok = issue_qkv(0, cur);
-      }
-      while (have && ok) {
-        // next valid unit of this CTA
-        bool have_next = false;
-        for (u += gridDim.x; u < units; u += gridDim.x)
-          if (decode_unit(p, u, true, &nxt)) { have_next = true; break; }
-        if (have_next) {
-          if (nxt.g != g_res) {
-            // W is read only by unit k's first MMA; wait for it before replacing W.
-            if (!tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim)) { ok = false; break; }
-            issue_w(nxt.g);
-            g_res = nxt.g;
-          }
-          if (!issue_qkv(k + 1, nxt)) { ok = false; break; }
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        Unit x;
+        if (!decode_unit(p, u, true, &x)) continue;
+        if (x.g != g_res) {
+          // W is read only by the first MMA of each unit: wait for the previous unit's
+          if (k >= 1 && !tc::mbar_wait(&sm.u_full, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+          tc::mbar_arrive_expect_tx(&sm.w_full, kWBytes);
+          tc::tma_load_2d(sm.w, &p.tm_w, &sm.w_full, 0, x.g * kD);
+          tc::tma_load_2d(sm.w + kWBytes / 2, &p.tm_w, &sm.w_full, 64, x.g * kD);
+          armed_w = w_loads & 1;
+          ++w_loads;
+          g_res = x.g;
         }
-        const int srow0 = (cur.slot * p.Hkv + cur.g) * kF;
-        for (int c = 0; c < kChunks; ++c, ++q) {
-          const int st = q % kStages, j = q / kStages;
-          if (j >= 1 && !tc::mbar_wait(&sm.s_empty[st], (j - 1) & 1, abort_flag, lim)) { ok = false; break; }
-          tc::mbar_arrive_expect_tx(&sm.s_full[st], kSBytes);
+        if (k >= 1 && !tc::mbar_wait(&sm.qk_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        tc::mbar_arrive_expect_tx(&sm.qk_full, kQBytes + kKBytes);
+        tc::tma_load_3d(sm.q, &p.tm_q, &sm.qk_full, 0, kG * x.g, x.lo);
+        tc::tma_load_3d(sm.q + kQBytes / 2, &p.tm_q, &sm.qk_full, 64, kG * x.g, x.lo);
+        tc::tma_load_3d(sm.k, &p.tm_k, &sm.qk_full, 0, x.g, x.lo);
+        tc::tma_load_3d(sm.k + kKBytes / 2, &p.tm_k, &sm.qk_full, 64, x.g, x.lo);
+        armed_qk = k & 1;
+        if (k >= 1 && !tc::mbar_wait(&sm.vz_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        tc::mbar_arrive_expect_tx(&sm.vz_full, kKBytes + kZBytes);
+        tc::tma_load_3d(sm.v, &p.tm_v, &sm.vz_full, 0, x.g, x.lo);
+        tc::tma_load_3d(sm.v + kKBytes / 2, &p.tm_v, &sm.vz_full, 64, x.g, x.lo);
+        tc::bulk_load(sm.z, p.Z + ((size_t)x.slot * p.Hkv + x.g) * kF, kZBytes, &sm.vz_full);
+        armed_vz = k & 1;
+        const int srow0 = (x.slot * p.Hkv + x.g) * kF;
+        for (int c = 0; c < kChunks; ++c) {
+          if (k >= 1 && !tc::mbar_wait(&sm.s_empty[c], (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+          tc::mbar_arrive_expect_tx(&sm.s_full[c], kSBytes);
 #pragma unroll
           for (int dq = 0; dq < 4; ++dq)
-            tc::tma_load_2d(sm.s[st] + dq * (kSBytes / 4), &p.tm_s, &sm.s_full[st], dq * 32,
+            tc::tma_load_2d(sm.s[c] + dq * (kSBytes / 4), &p.tm_s, &sm.s_full[c], dq * 32,
                             srow0 + c * kChunk);
-          armed_s[st] = j & 1;
+          armed_s[c] = k & 1;
         }
-        if (!ok) break;
-        cur = nxt;
-        have = have_next;
         ++k;
       }
       // Drain: every copy this thread started has landed before the CTA can exit.
-      const long long drain_lim = lim;
       volatile int never = 0;
-      for (int b = 0; b < 2; ++b)
-        if (armed_qkv[b] >= 0) tc::mbar_wait(&sm.qkv_full[b], armed_qkv[b], &never, drain_lim);
-      for (int s = 0; s < kStages; ++s)
-        if (armed_s[s] >= 0) tc::mbar_wait(&sm.s_full[s], armed_s[s], &never, drain_lim);
-      if (armed_w >= 0) tc::mbar_wait(&sm.w_full, armed_w, &never, drain_lim);
+      if (armed_qk >= 0) tc::mbar_wait(&sm.qk_full, armed_qk, &never, lim);
+      if (armed_vz >= 0) tc::mbar_wait(&sm.vz_full, armed_vz, &never, lim);
+      for (int c = 0; c < kStages; ++c)
+        if (armed_s[c] >= 0) tc::mbar_wait(&sm.s_full[c], armed_s[c], &never, lim);
+      if (armed_w >= 0) tc::mbar_wait(&sm.w_full, armed_w, &never, lim);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int k = 0, q = 0, g_res = -1;
+      int k = 0, g_res = -1;
       uint32_t w_seen = 0;
       bool ok = true;
       bool issued = false;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         Unit x;
         if (!decode_unit(p, u, false, &x)) continue;
-        const int buf = k & 1;
         if (x.g != g_res) {
           if (!tc::mbar_wait(&sm.w_full, w_seen & 1, abort_flag, lim)) { ok = false; break; }
           ++w_seen;
           g_res = x.g;
         }
-        if (!tc::mbar_wait(&sm.qkv_full[buf], (k >> 1) & 1, abort_flag, lim)) { ok = false; break; }
-        // the previous unit's MMAs read phi' from the columns u is about to overwrite
-        if (k >= 1 && !tc::mbar_wait(&sm.acc_full, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        if (!tc::mbar_wait(&sm.qk_full, k & 1, abort_flag, lim)) { ok = false; break; }
         tc::tc_fence_after();
-        const uint32_t qa = tc::smem_u32(sm.q[buf]);
+        const uint32_t qa = tc::smem_u32(sm.q);
         const uint32_t wa = tc::smem_u32(sm.w);
-        const uint32_t ka = tc::smem_u32(sm.k[buf]);
+        const uint32_t ka = tc::smem_u32(sm.k);
+        // u = Q W_g: the previous unit's u was consumed before its phi was published
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t a = tc::smem_desc(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
           const uint64_t b = tc::smem_desc(wa + kk * 2048, kWBytes / 2, 1024, tc::kSwizzle128B);
           tc::mma_bf16_ss(tbase + kColU, a, b, kIdQW, kk > 0);
         }
+        // s = Q K^T lands in the top phi' columns: the previous unit's state-read MMAs must be done
+        if (k >= 1 && !tc::mbar_wait(&sm.acc_full, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        tc::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t a = tc::smem_desc(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
@@ -268,21 +250,25 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
           tc::mma_bf16_ss(tbase + kColS, a, b, kIdQK, kk > 0);
         }
         tc::mma_commit(&sm.u_full);
+        tc::mma_commit(&sm.qk_empty);
         issued = true;
         if (!tc::mbar_wait(&sm.phi_ready, k & 1, abort_flag, lim)) { ok = false; break; }
+        if (!tc::mbar_wait(&sm.vz_full, k & 1, abort_flag, lim)) { ok = false; break; }
+        // P V overwrites the accumulator: the previous epilogue must have read it
         if (k >= 1 && !tc::mbar_wait(&sm.acc_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
         tc::tc_fence_after();
         const uint32_t pa = tc::smem_u32(sm.p);
-        const uint32_t va = tc::smem_u32(sm.v[buf]);
+        const uint32_t va = tc::smem_u32(sm.v);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
-          const uint64_t a = tc::smem_desc(pa + kk * 32, 16, 1024, tc::kSwizzle128B);
+          const uint64_t a = tc::smem_desc(pa + kk * 32, 16, 512, tc::kSwizzle64B);
           const uint64_t b = tc::smem_desc(va + kk * 2048, kKBytes / 2, 1024, tc::kSwizzle128B);
           tc::mma_bf16_ss(tbase + kColAcc, a, b, kIdPV, kk > 0);
         }
-        for (int c = 0; c < kChunks; ++c, ++q) {
-          const int st = q % kStages;
-          if (!tc::mbar_wait(&sm.s_full[st], (q / kStages) & 1, abort_flag, lim)) { ok = false; break; }
+        tc::mma_commit(&sm.vz_empty);
+        for (int c = 0; c < kChunks; ++c) {
+          const int st = c;
+          if (!tc::mbar_wait(&sm.s_full[st], k & 1, abort_flag, lim)) { ok = false; break; }
           tc::tc_fence_after();
           const uint32_t sa = tc::smem_u32(sm.s[st]);
 #pragma unroll
@@ -290,13 +276,12 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
             // MN-major tf32 operands use the 128-byte swizzle with 32-byte atoms: rows of 128 B,
             // 4-row K groups (SBO 512 B), d quarters 4 KiB apart (LBO).
             const uint64_t b = tc::smem_desc(sa + kk * 1024, kSBytes / 4, 512, tc::kSwizzle128BBase32B);
-            tc::mma_tf32_ts(tbase + kColAcc, tbase + kColU + c * kChunk + kk * 8, b, kIdPS, 1);
+            tc::mma_tf32_ts(tbase + kColAcc, tbase + kColPhi + c * kChunk + kk * 8, b, kIdPS, 1);
           }
           tc::mma_commit(&sm.s_empty[st]);
         }
         if (!ok) break;
         tc::mma_commit(&sm.acc_full);
-        tc::mma_commit(&sm.qkv_empty[buf]);
         ++k;
       }
       if (issued) {
@@ -308,21 +293,25 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
     }
   } else {
     // ------------------------------------------------------------ softmax / feature map / epilogue
-    const int wq = warp & 3;              // TMEM lane quarter this warp may access
-    const int row = wq * 32 + lane;       // tile row = 4 t + head-in-group
+    // Two threads per tile row: warps 2-5 take the softmax(u) half of phi and output columns
+    // [0, 64), warps 6-9 the softmax(-u) half and output columns [64, 128).
+    const int sw = warp - 2;                    // 0..7
+    const int half = sw >> 2;                   // 0: softmax(u), 1: softmax(-u)
+    const float sgn = half ? -1.f : 1.f;
+    const int wq = warp & 3;                    // TMEM lane quarter this warp may access
+    const int row = wq * 32 + lane;             // tile row = 4 t + head-in-group
     const int t = row >> 2, hl = row & 3;
     const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
     const float scale_log2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
     const float log2e = 1.4426950408889634f;
-    const int tid = threadIdx.x - 64;     // 0..127
+    const int tid = sw * 32 + lane;             // 0..255
     int k = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       Unit x;
       if (!decode_unit(p, u, false, &x)) continue;
-      const int buf = k & 1;
       const int h = kG * x.g + hl;
-      const bool valid = t < x.n;
       if (!tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim)) break;
+      if (!tc::mbar_wait(&sm.vz_full, k & 1, abort_flag, lim)) break;
       tc::tc_fence_after();
 
       // block softmax over the x.n keys of this request (bidirectional, no mask)
@@ -333,40 +322,60 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
 #pragma unroll
       for (int j = 0; j < 32; ++j)
         if (j < x.n) mraw = fmaxf(mraw, sv[j]);
-      // m (in log2 units of the scaled score), floored so e^{-m} stays finite
+      // m in log2 units of the scaled score, floored so e^{-m} stays finite
       const float m2 = fmaxf(mraw * scale_log2, -40.f * log2e);
       const float wgt = p.alpha ? 1.f / (1.f + expf(-p.alpha[h])) : 1.f;
       float den_sm = 0.f;
-      uint32_t packed[16];
+      if (half == 0) {
+        // P = w e^{s/sqrt d - m} in bf16; the denominator sums the rounded values P V uses
+        uint32_t packed[16];
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        float a0 = 0.f, a1 = 0.f;
-        if (j < x.n) a0 = wgt * exp2f(fmaf(sv[j], scale_log2, -m2));
-        if (j + 1 < x.n) a1 = wgt * exp2f(fmaf(sv[j + 1], scale_log2, -m2));
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
-        den_sm += __low2float(b2) + __high2float(b2);
-        packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
-      }
-      uint8_t* prow = sm.p + row * 128;
+        for (int j = 0; j < 32; j += 2) {
+          float a0 = 0.f, a1 = 0.f;
+          if (j < x.n) a0 = wgt * tc::ex2(fmaf(sv[j], scale_log2, -m2));
+          if (j + 1 < x.n) a1 = wgt * tc::ex2(fmaf(sv[j + 1], scale_log2, -m2));
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
+          den_sm += __low2float(b2) + __high2float(b2);
+          packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        // P row: 64 bytes, 16-byte chunk c stored at chunk c ^ ((row / 2) % 4) (64-byte swizzle)
+        uint8_t* prow = sm.p + row * 64;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint4 v4 = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v4;
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v4 = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+          *reinterpret_cast<uint4*>(prow + ((c ^ ((row >> 1) & 3)) << 4)) = v4;
+        }
       }
       if (x.n < kBlk) {
         // rows of V past the block belong to another request (or are zero fill): clear them
-        const int nz = (kBlk - x.n) * 2 * 8;  // 16-byte chunks over both d halves
-        for (int i = tid; i < nz; i += 128) {
-          const int half = i / ((kBlk - x.n) * 8), rem = i % ((kBlk - x.n) * 8);
+        const int per_half = (kBlk - x.n) * 8;  // 16-byte chunks per d half
+        for (int i = tid; i < 2 * per_half; i += 256) {
+          const int hh = i / per_half, rem = i % per_half;
           const int jr = x.n + rem / 8, ch = rem % 8;
-          *reinterpret_cast<uint4*>(sm.v[buf] + half * (kKBytes / 2) + jr * 128 + ch * 16) =
+          *reinterpret_cast<uint4*>(sm.v + hh * (kKBytes / 2) + jr * 128 + ch * 16) =
               make_uint4(0, 0, 0, 0);
         }
       }
       tc::fence_proxy_async_smem();
+      // every thread has read its scores before the softmax(-u) half overwrites their columns
+      tc::tc_fence_before();
+      tc::named_barrier_sync(1, 256);
+      tc::tc_fence_after();
 
-      // feature map on u = q W_g: pass 1 max/min, pass 2 exponentials and sums, pass 3 scale
-      float umax = -INFINITY, umin = INFINITY;
+      // this thread's half of the feature map: e = 2^{(sgn u - max sgn u) log2 e}
+      float ext = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < kFh / 32; ++c) {
+        float uv[32];
+        tc::tmem_ld32(tl + kColU + c * 32, uv);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ext = fmaxf(ext, sgn * uv[i]);
+      }
+      const float ext2 = ext * log2e;
+      const float slog2e = sgn * log2e;
+      float esum = 0.f, zsum = 0.f;
+      const float* zb = sm.z + half * kFh;
 #pragma unroll 1
       for (int c = 0; c < kFh / 32; ++c) {
         float uv[32];
@@ -374,70 +383,76 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
         tc::tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          umax = fmaxf(umax, uv[i]);
-          umin = fminf(umin, uv[i]);
+          const float e = tc::ex2(fmaf(uv[i], slog2e, -ext2));
+          uv[i] = e;
+          esum += e;
+          zsum = fmaf(e, zb[c * 32 + i], zsum);
         }
+        tc::tmem_st32(tl + kColPhi + half * kFh + c * 32, uv);
       }
-      const float mx2 = umax * log2e, mn2 = umin * log2e;
-      float sp = 0.f, sn = 0.f, zp = 0.f, zn = 0.f;
-      const float* zb = sm.z[buf];
+      tc::tmem_wait_st();
+      const float em = tc::ex2(-m2);
+      const float a = em / esum;
 #pragma unroll 1
       for (int c = 0; c < kFh / 32; ++c) {
-        float uv[32], en[32];
-        tc::tmem_ld32(tl + kColU + c * 32, uv);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float ep = exp2f(fmaf(uv[i], log2e, -mx2));
-          en[i] = exp2f(fmaf(-uv[i], log2e, mn2));
-          uv[i] = ep;
-          sp += ep;
-          sn += en[i];
-          zp = fmaf(ep, zb[c * 32 + i], zp);
-          zn = fmaf(en[i], zb[kFh + c * 32 + i], zn);
-        }
-        tc::tmem_st32(tl + kColU + c * 32, uv);
-        tc::tmem_st32(tl + kColU + kFh + c * 32, en);
-      }
-      tc::tmem_wait_st();
-      const float em = exp2f(-m2);
-      const float ap = em / sp, an = em / sn;
-#pragma unroll 1
-      for (int c = 0; c < kF / 32; ++c) {
         float ev[32];
-        tc::tmem_ld32(tl + kColU + c * 32, ev);
+        tc::tmem_ld32(tl + kColPhi + half * kFh + c * 32, ev);
         tc::tmem_wait_ld();
-        const float a = c < kFh / 32 ? ap : an;
 #pragma unroll
         for (int i = 0; i < 32; ++i) ev[i] *= a;
-        tc::tmem_st32(tl + kColU + c * 32, ev);
+        tc::tmem_st32(tl + kColPhi + half * kFh + c * 32, ev);
       }
       tc::tmem_wait_st();
-      const float den = den_sm + em * (zp / sp + zn / sn);
+      // shared denominator w sum_j P + e^{-m} (zsum_+/esum_+ + zsum_-/esum_-)
+      sm.red[half][row] = half == 0 ? den_sm + em * (zsum / esum) : em * (zsum / esum);
+      tc::named_barrier_sync(1, 256);
+      const float den = sm.red[0][row] + sm.red[1][row];
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.phi_ready);
 
-      // epilogue
+      // epilogue: this thread's 64 output columns
       if (!tc::mbar_wait(&sm.acc_full, k & 1, abort_flag, lim)) break;
       tc::tc_fence_after();
       const float inv = den != 0.f ? 1.f / den : 0.f;
-      __nv_bfloat16* orow = p.O + ((size_t)(x.lo + t) * p.Hq + h) * kD;
-#pragma unroll 1
-      for (int c = 0; c < kD / 32; ++c) {
-        float ov[32];
-        tc::tmem_ld32(tl + kColAcc + c * 32, ov);
+      float ov[64];
+      {
+        float a32[32], b32[32];
+        tc::tmem_ld32(tl + kColAcc + half * 64, a32);
+        tc::tmem_ld32(tl + kColAcc + half * 64 + 32, b32);
         tc::tmem_wait_ld();
-        if (valid) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 o4 = make_uint4(pack_bf16(ov[i] * inv, ov[i + 1] * inv),
-                                  pack_bf16(ov[i + 2] * inv, ov[i + 3] * inv),
-                                  pack_bf16(ov[i + 4] * inv, ov[i + 5] * inv),
-                                  pack_bf16(ov[i + 6] * inv, ov[i + 7] * inv));
-            *reinterpret_cast<uint4*>(orow + c * 32 + i) = o4;
+        for (int i = 0; i < 32; ++i) {
+          ov[i] = a32[i] * inv;
+          ov[32 + i] = b32[i] * inv;
+        }
+      }
+      // Coalesced store through this warp's 1 KiB of the (now idle) P buffer: 8 rows at a time
+      // are staged (16-byte chunk c of staged row r at chunk c ^ r), then each store
+      // instruction writes 4 rows x 128 contiguous bytes.
+      uint8_t* stg = sm.p + sw * 1024;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if ((lane >> 3) == j) {
+          const int rr = lane & 7;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 o4 = make_uint4(pack_bf16(ov[8 * c], ov[8 * c + 1]), pack_bf16(ov[8 * c + 2], ov[8 * c + 3]),
+                                        pack_bf16(ov[8 * c + 4], ov[8 * c + 5]), pack_bf16(ov[8 * c + 6], ov[8 * c + 7]));
+            *reinterpret_cast<uint4*>(stg + rr * 128 + ((c ^ rr) << 4)) = o4;
           }
         }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int rr = 4 * i + (lane >> 3), c = lane & 7;
+          const uint4 o4 = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((c ^ rr) << 4));
+          const int grow = wq * 32 + 8 * j + rr;       // tile row
+          const int gt = grow >> 2, ghl = grow & 3;
+          if (gt < x.n)
+            *reinterpret_cast<uint4*>(p.O + ((size_t)(x.lo + gt) * p.Hq + kG * x.g + ghl) * kD + half * 64 + c * 8) = o4;
+        }
+        __syncwarp();
       }
       tc::tc_fence_before();
       __syncwarp();
