@@ -446,13 +446,228 @@ def bench_decode(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ other workloads
+def _line(metric, value, unit, args, world, ms_step, higher, config, **extra):
+    d = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": higher,
+         "scaling": "weak", "vs_baseline": None, "data": "synthetic", "config": config}
+    d.update(extra)
+    return d
+
+
+def _roof(nbytes, ms, peaks, peak_src, kernel, flops=None):
+    achieved = nbytes / (ms / 1e3) / 1e9
+    r = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+         "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": nbytes,
+         "kernel": kernel}
+    if flops is not None:
+        r["flops_per_launch"] = flops
+    return r
+
+
+def bench_commit(args, world, rank, local):
+    """Block commit for 128 requests x 4 KV heads (d 128, F 256, 32-token blocks): S and Z
+    updated in place; 4 rotating state sets (75 MB each) keep L2 from holding them."""
+    from linear_attention_diffusion_hedgehog_b200 import bha
+
+    peaks, src = load_peaks()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(99 + rank)
+    dev, bf = torch.device("cuda"), torch.bfloat16
+    W = (torch.randn((HKV, D, F // 2), generator=gen, device=dev) / D ** 0.5).to(bf)
+    cu = torch.arange(0, (R + 1) * B, B, dtype=torch.int32, device=dev)
+    sets = [dict(K=torch.randn((R * B, HKV, D), generator=gen, device=dev).to(bf),
+                 V=torch.randn((R * B, HKV, D), generator=gen, device=dev).to(bf),
+                 S=torch.randn((R, HKV, F, D), generator=gen, device=dev),
+                 Z=torch.rand((R, HKV, F), generator=gen, device=dev) * 8) for _ in range(NSETS)]
+    stream = torch.cuda.Stream()
+    dims = bha.make_dims(R, HKV, HKV, D, F, B, R * B, R, bf)
+
+    def step(i):
+        s = sets[i % NSETS]
+        bha.commit_block(cu, s["K"], s["V"], W, s["S"], s["Z"], max_block=B, stream=stream)
+
+    ms = max_over_ranks(time_graphed(step, args.steps, args.warmup, world, stream), world)
+    if rank == 0:
+        ms_step = ms / args.steps
+        cfg = {"workload": "block commit: fold a 32-token block into S/Z for 128 requests x 4 KV "
+                           "heads, head dim 128, feature dim 256", "requests": R, "kv_heads": HKV,
+               "head_dim": D, "feature_dim": F, "block": B,
+               "l2": f"rotating {NSETS} state sets (~75 MB each)"}
+        print(json.dumps(_line("block-commit tokens/s (128 reqs x 4 KV heads)",
+                               R * B * world / (ms_step / 1e3), UNIT, args, world, ms_step, True, cfg,
+                               dtype="bf16 in, fp32 state", kernel_variant=bha.kernel_variant(dims, 2),
+                               roofline=_roof(commit_bytes(), ms_step, peaks, src, "commit",
+                                              flops=2 * R * HKV * B * (D * (F // 2) + F * D + F)),
+                               gpu_launches=args.steps)), flush=True)
+
+
+def bench_featuremap(args, world, rank, local):
+    """Standalone feature map phi(x) on the decode step's queries: x [4096, 16, 128] bf16 ->
+    phi [4096, 16, 256] fp32, 4 KV-head weight matrices; 2 rotating sets (84 MB each)."""
+    from linear_attention_diffusion_hedgehog_b200 import bha
+
+    peaks, src = load_peaks()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7 + rank)
+    dev, bf = torch.device("cuda"), torch.bfloat16
+    W = (torch.randn((HKV, D, F // 2), generator=gen, device=dev) / D ** 0.5).to(bf)
+    sets = [dict(x=torch.randn((R * B, HQ, D), generator=gen, device=dev).to(bf),
+                 o=torch.empty((R * B, HQ, F), device=dev)) for _ in range(2)]
+    stream = torch.cuda.Stream()
+
+    def step(i):
+        s = sets[i % 2]
+        bha.featuremap(s["x"], W, out=s["o"], stream=stream)
+
+    ms = max_over_ranks(time_graphed(step, args.steps, args.warmup, world, stream), world)
+    if rank == 0:
+        ms_step = ms / args.steps
+        rows = R * B * HQ
+        nbytes = rows * D * 2 + rows * F * 4 + HKV * D * (F // 2) * 2
+        cfg = {"workload": "feature map phi(x) of 4096 tokens x 16 heads, head dim 128, feature dim "
+                           "256, fp32 output", "tokens": R * B, "heads": HQ, "head_dim": D,
+               "feature_dim": F, "l2": "2 rotating sets (~84 MB each)"}
+        print(json.dumps(_line("feature-map rows/s", rows * world / (ms_step / 1e3), "rows/s", args,
+                               world, ms_step, True, cfg, dtype="bf16 in, f32 out",
+                               roofline=_roof(nbytes, ms_step, peaks, src, "featuremap",
+                                              flops=2 * rows * D * (F // 2)),
+                               gpu_launches=args.steps)), flush=True)
+
+
+def bench_sweep(args, world, rank, local):
+    """Decode step vs the full-prefix softmax teacher at 64 requests (16 query / 4 KV heads,
+    head dim 128, 32-token blocks) over prefixes of 512 .. 32768 tokens.  The hybrid reads only
+    the fixed-size states; the teacher reads a bf16 KV cache of prefix + block tokens."""
+    from linear_attention_diffusion_hedgehog_b200 import bha
+
+    peaks, src = load_peaks()
+    dev, bf = torch.device("cuda"), torch.bfloat16
+    Rs = 64
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5 + rank)
+    W, cu, hsets = make_decode_sets(gen, nsets=NSETS, R=Rs, prefix=0, states_from_commits=False)
+    for s in hsets:
+        s["S"].normal_(generator=gen)
+        s["Z"].uniform_(0.5, 1.5, generator=gen)
+    stream = torch.cuda.Stream()
+    steps = args.steps
+
+    def hstep(i):
+        s = hsets[i % NSETS]
+        bha.hybrid_attn(cu, s["Q"], s["K"], s["V"], s["S"], s["Z"], W, max_block=B, out=s["O"],
+                        stream=stream)
+
+    h_ms = max_over_ranks(time_graphed(hstep, steps, args.warmup, world, stream), world) / steps
+    out = []
+    for P in (512, 2048, 8192, 32768):
+        L = P + B
+        cap = L
+        nsets = max(1, min(NSETS, int(np.ceil(400e6 / (Rs * HKV * L * D * 2 * 2)))))
+        tsets = []
+        for _ in range(nsets):
+            Kc = torch.randn((Rs, HKV, cap, D), generator=gen, device=dev).to(bf)
+            Vc = torch.randn((Rs, HKV, cap, D), generator=gen, device=dev).to(bf)
+            tsets.append(dict(Kc=Kc, Vc=Vc, Q=hsets[0]["Q"], O=torch.empty_like(hsets[0]["O"])))
+        kv_len = torch.full((Rs,), L, dtype=torch.int32, device=dev)
+        ws_bytes = bha.full_prefix_workspace_bytes(Rs, HQ, HKV, D, B, Rs * B, cap)
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+
+        def tstep(i):
+            s = tsets[i % nsets]
+            bha.full_prefix_attn(cu, kv_len, s["Q"], s["Kc"], s["Vc"], max_block=B, workspace=ws,
+                                 out=s["O"], stream=stream)
+
+        tsteps = max(3, min(steps, int(2e5 // max(P, 1))))
+        t_ms = max_over_ranks(time_graphed(tstep, tsteps, args.warmup, world, stream), world) / tsteps
+        del tsets
+        torch.cuda.empty_cache()
+        hb = step_bytes(R=Rs)
+        tb = teacher_bytes(Rs, HQ, HKV, D, B, P)
+        out.append({"prefix": P, "hybrid_ms": h_ms, "teacher_ms": t_ms, "speedup": t_ms / h_ms,
+                    "hybrid_hbm_frac": hb / (h_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                    "teacher_hbm_frac": tb / (t_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                    "teacher_steps": tsteps})
+    if rank == 0:
+        cfg = {"workload": "hybrid decode step (states only) vs full-prefix softmax teacher, 64 "
+                           "requests, 16 query / 4 KV heads, head dim 128, 32-token blocks",
+               "requests": Rs, "prefixes": [o["prefix"] for o in out]}
+        print(json.dumps(_line("hybrid vs teacher per-block latency over prefix length",
+                               out[-1]["speedup"], "x (teacher/hybrid at 32K prefix)", args, world,
+                               h_ms, True, cfg, dtype="bf16", sweep=out)), flush=True)
+
+
+def bench_cycle(args, world, rank, local):
+    """Ragged serving mix: 128 requests with prefix lengths uniform on {0, 32, ..., 8192},
+    32-token blocks, 6 hybrid layers (16 query / 4 KV heads, head dim 128, F 256, independent
+    W), 8 denoising steps per block then a commit of every layer, captured as one CUDA graph.
+    A step of this workload is one whole block cycle."""
+    from linear_attention_diffusion_hedgehog_b200 import bha, inputs
+
+    peaks, src = load_peaks()
+    dev, bf = torch.device("cuda"), torch.bfloat16
+    layers, nsteps = 6, 8
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(11 + rank)
+    plen = inputs.ragged_prefix_lengths(R, seed=5)
+    cu = torch.arange(0, (R + 1) * B, B, dtype=torch.int32, device=dev)
+    Ws = [(torch.randn((HKV, D, F // 2), generator=gen, device=dev) / D ** 0.5).to(bf)
+          for _ in range(layers)]
+    Ss = [torch.zeros((R, HKV, F, D), device=dev) for _ in range(layers)]
+    Zs = [torch.zeros((R, HKV, F), device=dev) for _ in range(layers)]
+    # prefix states: one commit call per 128-token slice of each request's prefix
+    for l in range(layers):
+        for j in range(0, int(plen.max()), 128):
+            lens = np.clip(plen - j, 0, 128)
+            if lens.sum() == 0:
+                break
+            cuj = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+            T = int(lens.sum())
+            Kb = torch.randn((T, HKV, D), generator=gen, device=dev).to(bf)
+            Vb = torch.randn((T, HKV, D), generator=gen, device=dev).to(bf)
+            bha.commit_block(cuj, Kb, Vb, Ws[l], Ss[l], Zs[l], max_block=128)
+    acts = [[dict(Q=torch.randn((R * B, HQ, D), generator=gen, device=dev).to(bf),
+                  K=torch.randn((R * B, HKV, D), generator=gen, device=dev).to(bf),
+                  V=torch.randn((R * B, HKV, D), generator=gen, device=dev).to(bf))
+             for _ in range(layers)] for _ in range(nsteps)]
+    O = torch.empty((R * B, HQ, D), device=dev, dtype=bf)
+    stream = torch.cuda.Stream()
+
+    def cycle(i):
+        for st in range(nsteps):
+            for l in range(layers):
+                a = acts[st][l]
+                bha.hybrid_attn(cu, a["Q"], a["K"], a["V"], Ss[l], Zs[l], Ws[l], max_block=B,
+                                out=O, stream=stream)
+        for l in range(layers):
+            a = acts[nsteps - 1][l]
+            bha.commit_block(cu, a["K"], a["V"], Ws[l], Ss[l], Zs[l], max_block=B, stream=stream)
+
+    ms = max_over_ranks(time_graphed(cycle, args.steps, args.warmup, world, stream), world)
+    if rank == 0:
+        ms_cycle = ms / args.steps
+        nbytes = nsteps * layers * step_bytes() + layers * commit_bytes()
+        cfg = {"workload": "ragged serving mix: 128 requests, prefixes uniform on {0,32,...,8192}, "
+                           "32-token blocks, 6 hybrid layers, 8 denoising steps then a commit per "
+                           "block cycle (one CUDA graph)", "requests": R, "layers": layers,
+               "steps_per_block": nsteps, "prefix_mean": float(plen.mean())}
+        print(json.dumps(_line("serving-cycle tokens/s per denoise step (6 hybrid layers)",
+                               nsteps * R * B * world / (ms_cycle / 1e3), UNIT, args, world,
+                               ms_cycle, True, cfg, dtype="bf16 in, fp32 state",
+                               roofline=_roof(nbytes, ms_cycle, peaks, src, "block cycle"),
+                               committed_tokens_per_s=R * B * world / (ms_cycle / 1e3),
+                               gpu_launches=args.steps * (nsteps * layers + layers))), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "commit", "sweep", "cycle"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "commit", "featuremap", "sweep", "cycle"],
+                    default="decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
@@ -465,7 +680,8 @@ def main():
         if args.workload == "decode":
             bench_decode(args, world, rank, local)
         else:
-            raise SystemExit(f"workload {args.workload!r} is not available yet")
+            {"commit": bench_commit, "featuremap": bench_featuremap, "sweep": bench_sweep,
+             "cycle": bench_cycle}[args.workload](args, world, rank, local)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -69,6 +69,17 @@ int bha_kernel_variant(const bha_dims* dims, int32_t which) {
     a.num_slots = dims->num_slots;
     return bha::hybrid_tc_supports(a, bf16) ? 1 : 0;
   }
+  if (which == 2) {
+    bha::CommitArgs c{};
+    c.R = dims->num_requests;
+    c.Hkv = dims->num_kv_heads;
+    c.d = dims->head_dim;
+    c.F = dims->feature_dim;
+    c.Bmax = dims->max_block;
+    c.T = dims->total_tokens;
+    c.num_slots = dims->num_slots;
+    return bha::commit_tc_supports(c, bf16) ? 1 : 0;
+  }
   return 0;
 }
 
@@ -131,8 +142,10 @@ int bha_commit_block(const bha_dims* dims, const int32_t* cu_blk, const int32_t*
   bha::CommitArgs a{cu_blk, state_slot, K, V, W, S, Z, dev_err, dims->num_requests,
                     dims->num_kv_heads, dims->head_dim, dims->feature_dim, dims->max_block,
                     dims->total_tokens, dims->num_slots};
-  return launch_status(
-      bha::launch_commit_simt(a, dims->act_dtype == BHA_BF16, static_cast<cudaStream_t>(stream)));
+  const bool bf16 = dims->act_dtype == BHA_BF16;
+  if (bha::commit_tc_supports(a, bf16))
+    return launch_status(bha::launch_commit_tc(a, static_cast<cudaStream_t>(stream)));
+  return launch_status(bha::launch_commit_simt(a, bf16, static_cast<cudaStream_t>(stream)));
 }
 
 size_t bha_full_prefix_workspace_bytes(const bha_dims* dims, int64_t kv_capacity) {

@@ -1,0 +1,431 @@
+// Tensor-core block commit for sm_100a (bf16 activations, d = 128, F = 256, blocks of up
+// to 32 tokens).
+//
+// Source: "Retrofitting Linear Attention into Diffusion Language Models", §3.1, the commit
+// of a finished block:  S_n = S_{n-1} + sum_{t in B_n} phi(k_t) v_t^T,  Z_n = Z_{n-1} +
+// sum_{t in B_n} phi(k_t),  phi(k) = [softmax(kW), softmax(-kW)].
+//
+// Work unit: four requests that share KV head g (their 4 x 32 key rows form one 128-row
+// MMA tile for u = K W_g).  Per unit:
+//   u     = K W_g                 bf16 MMA, M 128 (4 requests x 32 tokens), N 128, K 128
+//   phi   = [softmax(u), softmax(-u)] per row on CUDA cores (two threads per row), rounded
+//           to bf16 into shared memory as the B operand of the next MMA; rows past a
+//           request's block are zero, so they add nothing
+//   dZ    = column sums of the bf16 phi over each request's tokens (CUDA cores)
+//   dS^T  = V_r^T phi_r           bf16 MMA per request, M 128 (d), N 256 (F), K 32 (tokens)
+//                                 into one of two TMEM buffers
+//   S += dS, Z += dZ               fp32 read-modify-write by 8 warps: TMEM lane = d, so each
+//                                 warp instruction reads or writes one whole 128-byte line
+//                                 of a row of S; the other buffer's MMA overlaps it.
+// Computing dS transposed (lanes = d) is what makes the state update coalesced without
+// staging it through shared memory.
+//
+// Roles (320 threads): warp 0 TMA producer (K, V, W), warp 1 TMEM owner and MMA issuer,
+// warps 2-9 feature map, dZ and the state update.  Every wait is bounded; on expiry the CTA
+// records BHA_ERR_TIMEOUT, drains its copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_util.cuh"
+
+namespace bha {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kF = 256;
+constexpr int kFh = 128;
+constexpr int kBlk = 32;
+constexpr int kReq = 4;          // requests per unit
+constexpr int kM = kReq * kBlk;  // 128 key rows
+constexpr int kThreads = 320;
+
+constexpr uint32_t kKBytes = kM * kD * 2;        // 32 KiB: [d half][128 rows][128 B]
+constexpr uint32_t kWBytes = kD * kFh * 2;       // 32 KiB: [f half][128 rows of d][128 B]
+constexpr uint32_t kVReqBytes = kBlk * kD * 2;   // 8 KiB per request: [d half][32 rows][128 B]
+constexpr uint32_t kPhiReqBytes = kBlk * kF * 2; // 16 KiB per request: [f quarter][32 rows][128 B]
+
+constexpr uint32_t kColU = 0;     // u (128 columns), inside dS buffer 0
+constexpr uint32_t kColD0 = 0;    // dS^T buffers: 256 columns each
+constexpr uint32_t kColD1 = 256;
+constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t kIdKW = tc::instr_desc(1, 0, 1, kM, kFh);   // A K-major, B MN-major
+constexpr uint32_t kIdVP = tc::instr_desc(1, 1, 1, kD, kF);    // A MN-major (V^T), B MN-major
+
+struct __align__(1024) Smem {
+  uint8_t k[kKBytes];
+  uint8_t w[kWBytes];
+  uint8_t v[kReq][kVReqBytes];
+  uint8_t phi[kReq][kPhiReqBytes];
+  float dz[kReq][kF];
+  uint64_t k_full, k_empty, v_full, v_empty, w_full, u_full, phi_ready;
+  uint64_t d_full[2], d_empty[2], drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory budget");
+
+struct Req {
+  int lo, n, slot;  // n = 0: absent (no request, empty block or invalid)
+};
+
+// The four requests of unit (j0, g); every role decodes them identically.
+__device__ __forceinline__ void decode_unit(const TcCommitParams& p, int j0, bool report,
+                                            Req (&rq)[kReq]) {
+#pragma unroll
+  for (int j = 0; j < kReq; ++j) {
+    rq[j].n = 0;
+    rq[j].lo = 0;
+    rq[j].slot = 0;
+    const int r = j0 + j;
+    if (r >= p.R) continue;
+    RowRange rr;
+    if (!request_rows(p.cu_blk, r, p.T, p.Bmax, p.dev_err, report, &rr)) continue;
+    int slot;
+    if (!request_slot(p.state_slot, r, p.num_slots, p.dev_err, report, &slot)) continue;
+    rq[j].lo = rr.lo;
+    rq[j].n = rr.n;
+    rq[j].slot = slot;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_constant__ TcCommitParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &sm.abort_flag;
+  const long long lim = p.wait_limit;
+  const int groups = (p.R + kReq - 1) / kReq;
+  const int units = groups * p.Hkv;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&sm.k_full, 1);
+    tc::mbar_init(&sm.k_empty, 1);
+    tc::mbar_init(&sm.v_full, 1);
+    tc::mbar_init(&sm.v_empty, 1);
+    tc::mbar_init(&sm.w_full, 1);
+    tc::mbar_init(&sm.u_full, 1);
+    tc::mbar_init(&sm.phi_ready, 8);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&sm.d_full[i], 1);
+      tc::mbar_init(&sm.d_empty[i], 8);
+    }
+    tc::mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::prefetch_tensormap(&p.tm_k);
+    tc::prefetch_tensormap(&p.tm_v);
+    tc::prefetch_tensormap(&p.tm_w);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&sm.tmem_base, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int k = 0, g_res = -1;
+      uint32_t w_loads = 0;
+      int armed_k = -1, armed_v = -1, armed_w = -1;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const int g = u % p.Hkv, j0 = (u / p.Hkv) * kReq;
+        Req rq[kReq];
+        decode_unit(p, j0, true, rq);
+        int nreq = 0;
+#pragma unroll
+        for (int j = 0; j < kReq; ++j) nreq += rq[j].n > 0;
+        if (nreq == 0) continue;
+        if (g != g_res) {
+          if (k >= 1 && !tc::mbar_wait(&sm.u_full, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+          tc::mbar_arrive_expect_tx(&sm.w_full, kWBytes);
+          tc::tma_load_2d(sm.w, &p.tm_w, &sm.w_full, 0, g * kD);
+          tc::tma_load_2d(sm.w + kWBytes / 2, &p.tm_w, &sm.w_full, 64, g * kD);
+          armed_w = w_loads & 1;
+          ++w_loads;
+          g_res = g;
+        }
+        if (k >= 1 && !tc::mbar_wait(&sm.k_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        tc::mbar_arrive_expect_tx(&sm.k_full, nreq * 2 * (kBlk * 64 * 2));
+#pragma unroll
+        for (int j = 0; j < kReq; ++j) {
+          if (rq[j].n == 0) continue;
+          tc::tma_load_3d(sm.k + j * kBlk * 128, &p.tm_k, &sm.k_full, 0, g, rq[j].lo);
+          tc::tma_load_3d(sm.k + kKBytes / 2 + j * kBlk * 128, &p.tm_k, &sm.k_full, 64, g, rq[j].lo);
+        }
+        armed_k = k & 1;
+        if (k >= 1 && !tc::mbar_wait(&sm.v_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        tc::mbar_arrive_expect_tx(&sm.v_full, nreq * kVReqBytes);
+#pragma unroll
+        for (int j = 0; j < kReq; ++j) {
+          if (rq[j].n == 0) continue;
+          tc::tma_load_3d(sm.v[j], &p.tm_v, &sm.v_full, 0, g, rq[j].lo);
+          tc::tma_load_3d(sm.v[j] + kVReqBytes / 2, &p.tm_v, &sm.v_full, 64, g, rq[j].lo);
+        }
+        armed_v = k & 1;
+        ++k;
+      }
+      volatile int never = 0;
+      if (armed_k >= 0) tc::mbar_wait(&sm.k_full, armed_k, &never, lim);
+      if (armed_v >= 0) tc::mbar_wait(&sm.v_full, armed_v, &never, lim);
+      if (armed_w >= 0) tc::mbar_wait(&sm.w_full, armed_w, &never, lim);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int k = 0, g_res = -1, rc = 0;
+      uint32_t w_seen = 0;
+      int uses[2] = {0, 0};  // completed-or-issued uses of each dS buffer
+      bool ok = true, issued = false;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const int g = u % p.Hkv, j0 = (u / p.Hkv) * kReq;
+        Req rq[kReq];
+        decode_unit(p, j0, false, rq);
+        int nreq = 0;
+#pragma unroll
+        for (int j = 0; j < kReq; ++j) nreq += rq[j].n > 0;
+        if (nreq == 0) continue;
+        if (g != g_res) {
+          if (!tc::mbar_wait(&sm.w_full, w_seen & 1, abort_flag, lim)) { ok = false; break; }
+          ++w_seen;
+          g_res = g;
+        }
+        if (!tc::mbar_wait(&sm.k_full, k & 1, abort_flag, lim)) { ok = false; break; }
+        // u lands in dS buffer 0: its last state update must have read it
+        if (uses[0] >= 1 && !tc::mbar_wait(&sm.d_empty[0], (uses[0] - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        tc::tc_fence_after();
+        const uint32_t ka = tc::smem_u32(sm.k), wa = tc::smem_u32(sm.w);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint64_t a = tc::smem_desc(ka + (kk >> 2) * (kKBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
+          const uint64_t b = tc::smem_desc(wa + kk * 2048, kWBytes / 2, 1024, tc::kSwizzle128B);
+          tc::mma_bf16_ss(tbase + kColU, a, b, kIdKW, kk > 0);
+        }
+        tc::mma_commit(&sm.u_full);
+        tc::mma_commit(&sm.k_empty);
+        issued = true;
+        if (!tc::mbar_wait(&sm.phi_ready, k & 1, abort_flag, lim)) { ok = false; break; }
+        if (!tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim)) { ok = false; break; }
+        for (int j = 0; j < kReq && ok; ++j) {
+          if (rq[j].n == 0) continue;
+          const int b = rc & 1;
+          if (uses[b] >= 1 && !tc::mbar_wait(&sm.d_empty[b], (uses[b] - 1) & 1, abort_flag, lim)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t va = tc::smem_u32(sm.v[j]), pa = tc::smem_u32(sm.phi[j]);
+#pragma unroll
+          for (int kk = 0; kk < kBlk / 16; ++kk) {
+            // A = V^T (M = d, K = tokens), MN-major: d halves 4 KiB apart, 8-token groups 1 KiB
+            const uint64_t a = tc::smem_desc(va + kk * 2048, kVReqBytes / 2, 1024, tc::kSwizzle128B);
+            // B = phi (K = tokens, N = F), MN-major: F quarters 4 KiB apart
+            const uint64_t bd = tc::smem_desc(pa + kk * 2048, kPhiReqBytes / 4, 1024, tc::kSwizzle128B);
+            tc::mma_bf16_ss(tbase + (b ? kColD1 : kColD0), a, bd, kIdVP, kk > 0);
+          }
+          tc::mma_commit(&sm.d_full[b]);
+          ++uses[b];
+          ++rc;
+        }
+        if (!ok) break;
+        tc::mma_commit(&sm.v_empty);
+        ++k;
+      }
+      if (issued) {
+        volatile int never = 0;
+        tc::mma_commit(&sm.drain);
+        tc::mbar_wait(&sm.drain, 0, &never, lim);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ feature map, dZ, state update
+    const int sw = warp - 2;          // 0..7
+    const int half = sw >> 2;         // feature-map half / F half of the state update
+    const float sgn = half ? -1.f : 1.f;
+    const int wq = warp & 3;          // TMEM lane quarter
+    const int row = wq * 32 + lane;   // key row = 32 j + t during the feature map; d afterwards
+    const int tid = sw * 32 + lane;   // 0..255
+    const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
+    const float log2e = 1.4426950408889634f;
+    int k = 0, rc = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      const int g = u % p.Hkv, j0 = (u / p.Hkv) * kReq;
+      Req rq[kReq];
+      decode_unit(p, j0, false, rq);
+      int nreq = 0;
+#pragma unroll
+      for (int j = 0; j < kReq; ++j) nreq += rq[j].n > 0;
+      if (nreq == 0) continue;
+      if (!tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim)) break;
+      if (!tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim)) break;
+      tc::tc_fence_after();
+      // ---- this thread's half of phi for key row `row`, rounded to bf16
+      const int jr = row >> 5, t = row & 31;
+      const bool live = t < rq[jr].n;
+      float e[kFh];
+      {
+        float ext = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kFh / 32; ++c) {
+          float uv[32];
+          tc::tmem_ld32(tl + kColU + c * 32, uv);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            e[c * 32 + i] = sgn * uv[i];
+            ext = fmaxf(ext, e[c * 32 + i]);
+          }
+        }
+        float esum = 0.f;
+#pragma unroll
+        for (int i = 0; i < kFh; ++i) {
+          e[i] = tc::ex2((e[i] - ext) * log2e);
+          esum += e[i];
+        }
+        const float inv = 1.f / esum;
+        // phi_j as the B operand: F quarter a = 2 half + f / 64, row t, 16-byte chunk
+        // (f % 64) / 8 stored at chunk ^ (t % 8).  Rows past the block are written as zeros
+        // (selected, not multiplied, so stale shared memory cannot inject a NaN).
+        uint8_t* base = sm.phi[jr] + (2 * half) * (kPhiReqBytes / 4) + t * 128;
+#pragma unroll
+        for (int c = 0; c < kFh / 8; ++c) {
+          uint4 v4 = make_uint4(0, 0, 0, 0);
+          if (live)
+            v4 = make_uint4(pack_bf16(e[8 * c] * inv, e[8 * c + 1] * inv),
+                            pack_bf16(e[8 * c + 2] * inv, e[8 * c + 3] * inv),
+                            pack_bf16(e[8 * c + 4] * inv, e[8 * c + 5] * inv),
+                            pack_bf16(e[8 * c + 6] * inv, e[8 * c + 7] * inv));
+          const int quarter = c >> 3, ch = c & 7;
+          *reinterpret_cast<uint4*>(base + quarter * (kPhiReqBytes / 4) + ((ch ^ (t & 7)) << 4)) = v4;
+        }
+      }
+      // rows of V past a request's block (or of an absent request) are cleared, so that
+      // nothing from another request can leak in through 0 x (non-finite) products
+#pragma unroll
+      for (int j = 0; j < kReq; ++j) {
+        const int n = rq[j].n;
+        if (n >= kBlk || n == 0) continue;
+        const int per_half = (kBlk - n) * 8;
+        for (int i = tid; i < 2 * per_half; i += 256) {
+          const int hh = i / per_half, rem = i % per_half;
+          *reinterpret_cast<uint4*>(sm.v[j] + hh * (kVReqBytes / 2) + (n + rem / 8) * 128 + (rem % 8) * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
+      }
+      tc::tc_fence_before();
+      tc::named_barrier_sync(1, 256);
+      tc::tc_fence_after();
+      // ---- dZ[j][f] = sum over the block's tokens of the bf16 phi (thread tid owns f = tid)
+      {
+        const int f = tid, quarter = f >> 6, ch = (f & 63) >> 3, w8 = f & 7;
+#pragma unroll
+        for (int j = 0; j < kReq; ++j) {
+          float acc = 0.f;
+          if (rq[j].n > 0) {
+            const uint8_t* base = sm.phi[j] + quarter * (kPhiReqBytes / 4);
+            for (int tt = 0; tt < rq[j].n; ++tt) {
+              const __nv_bfloat16 vb =
+                  *reinterpret_cast<const __nv_bfloat16*>(base + tt * 128 + ((ch ^ (tt & 7)) << 4) + w8 * 2);
+              acc += __bfloat162float(vb);
+            }
+          }
+          sm.dz[j][f] = acc;
+        }
+      }
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sm.phi_ready);
+
+      // ---- state update per request: S[f][d] += dS^T[d][f], Z[f] += dZ[f]
+      const int d = row;  // TMEM lane = d
+      for (int j = 0; j < kReq; ++j) {
+        if (rq[j].n == 0) continue;
+        const int b = rc & 1;
+        if (!tc::mbar_wait(&sm.d_full[b], (rc >> 1) & 1, abort_flag, lim)) { k = -1; break; }
+        tc::tc_fence_after();
+        float* Sg = p.S + ((size_t)rq[j].slot * p.Hkv + g) * kF * kD;
+        const uint32_t col0 = (b ? kColD1 : kColD0) + half * kFh;
+#pragma unroll 1
+        for (int fc = 0; fc < kFh / 32; ++fc) {
+          float dv[32], sv[32];
+          tc::tmem_ld32(tl + col0 + fc * 32, dv);
+          const int f0 = half * kFh + fc * 32;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sv[i] = Sg[(size_t)(f0 + i) * kD + d];
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) Sg[(size_t)(f0 + i) * kD + d] = sv[i] + dv[i];
+        }
+        float* Zg = p.Z + ((size_t)rq[j].slot * p.Hkv + g) * kF;
+        Zg[tid] += sm.dz[j][tid];
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&sm.d_empty[b]);
+        ++rc;
+      }
+      if (k < 0) break;
+      ++k;
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);
+  if (threadIdx.x == 0 && sm.abort_flag) set_error(p.dev_err, BHA_ERR_TIMEOUT);
+}
+
+}  // namespace
+
+bool commit_tc_supports(const CommitArgs& a, bool act_bf16) {
+  return act_bf16 && a.d == kD && a.F == kF && a.Bmax <= kBlk &&
+         (long long)a.num_slots * a.Hkv * kF * kD < (1ll << 40);
+}
+
+cudaError_t launch_commit_tc(const CommitArgs& a, cudaStream_t st) {
+  TcCommitParams p;
+  const uint64_t T = (uint64_t)a.T;
+  {
+    const uint64_t dims[3] = {kD, (uint64_t)a.Hkv, T};
+    const uint64_t strides[2] = {kD * 2, (uint64_t)a.Hkv * kD * 2};
+    const uint32_t box[3] = {64, 1, kBlk};
+    if (!make_tensor_map(&p.tm_k, false, 3, a.K, dims, strides, box, false)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&p.tm_v, false, 3, a.V, dims, strides, box, false)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[2] = {kFh, (uint64_t)a.Hkv * kD};
+    const uint64_t strides[1] = {kFh * 2};
+    const uint32_t box[2] = {64, kD};
+    if (!make_tensor_map(&p.tm_w, false, 2, a.W, dims, strides, box, false)) return cudaErrorInvalidValue;
+  }
+  p.cu_blk = a.cu_blk;
+  p.state_slot = a.state_slot;
+  p.S = a.S;
+  p.Z = a.Z;
+  p.dev_err = a.dev_err;
+  p.R = a.R;
+  p.Hkv = a.Hkv;
+  p.T = a.T;
+  p.Bmax = a.Bmax;
+  p.num_slots = a.num_slots;
+  p.wait_limit = 2000000000ll;
+  const int units = ((a.R + kReq - 1) / kReq) * a.Hkv;
+  int nsm = device_sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
+  int grid = nsm;
+  if (a.Hkv <= nsm) grid = (nsm / a.Hkv) * a.Hkv;
+  if (grid > units) grid = units;
+  const size_t smem = sizeof(Smem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(commit_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  commit_tc_kernel<<<grid, kThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace bha

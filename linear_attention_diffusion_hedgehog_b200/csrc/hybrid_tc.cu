@@ -107,11 +107,6 @@ __device__ __forceinline__ bool decode_unit(const TcHybridParams& p, int u, bool
   return request_slot(p.state_slot, x->r, p.num_slots, p.dev_err, report, &x->slot);
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
-
 __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_constant__ TcHybridParams p) {
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));

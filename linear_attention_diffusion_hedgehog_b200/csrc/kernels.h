@@ -63,6 +63,18 @@ struct TcHybridParams {
   long long wait_limit;  // SM cycles a bounded wait may spin before giving up
 };
 
+// Parameters of the tensor-core block-commit kernel (commit_tc.cu).
+struct TcCommitParams {
+  CUtensorMap tm_k, tm_v, tm_w;
+  const int32_t* cu_blk;
+  const int32_t* state_slot;
+  float* S;
+  float* Z;
+  int32_t* dev_err;
+  int R, Hkv, T, Bmax, num_slots;
+  long long wait_limit;
+};
+
 // host helpers shared by the tensor-core launchers (hybrid_tc.cu)
 bool make_tensor_map(CUtensorMap* m, bool f32, int rank, const void* base, const uint64_t* dims,
                      const uint64_t* strides_bytes, const uint32_t* box, bool swizzle_atom32);
@@ -71,6 +83,8 @@ int device_sm_count();
 // tensor-core kernels
 bool hybrid_tc_supports(const HybridArgs& a, bool act_bf16);
 cudaError_t launch_hybrid_tc(const HybridArgs& a, cudaStream_t st);
+bool commit_tc_supports(const CommitArgs& a, bool act_bf16);
+cudaError_t launch_commit_tc(const CommitArgs& a, cudaStream_t st);
 
 // generic CUDA-core kernels (simt.cu)
 bool simt_supports(int d, int F, int Bmax);

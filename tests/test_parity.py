@@ -267,6 +267,8 @@ def test_tensor_core_path_is_taken_for_the_serving_shape():
     assert bha.kernel_variant(d, 1) == 1
     d32 = bha.make_dims(128, 16, 4, 128, 256, 32, 4096, 128, torch.float32)
     assert bha.kernel_variant(d32, 1) == 0   # fp32 activations take the fp32 CUDA-core path
+    assert bha.kernel_variant(d, 2) == 1     # block commit on tensor cores
+    assert bha.kernel_variant(d32, 2) == 0
 
 
 def test_linear_branch_dominant_states():
