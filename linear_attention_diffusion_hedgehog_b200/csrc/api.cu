@@ -30,6 +30,18 @@ int check_dims(const bha_dims* dm) {
 bool tensor_ok(const void* p) { return p != nullptr && aligned(p, 16); }
 bool index_ok(const void* p) { return p != nullptr && aligned(p, 4); }
 
+bha::FullPrefixArgs full_args(const bha_dims* dims, int64_t kv_capacity) {
+  bha::FullPrefixArgs a{};
+  a.kv_capacity = kv_capacity;
+  a.R = dims->num_requests;
+  a.Hq = dims->num_q_heads;
+  a.Hkv = dims->num_kv_heads;
+  a.d = dims->head_dim;
+  a.Bmax = dims->max_block;
+  a.T = dims->total_tokens;
+  return a;
+}
+
 int launch_status(cudaError_t e) {
   if (e == cudaSuccess) return BHA_OK;
   return BHA_ERR_CUDA;
@@ -80,6 +92,7 @@ int bha_kernel_variant(const bha_dims* dims, int32_t which) {
     c.num_slots = dims->num_slots;
     return bha::commit_tc_supports(c, bf16) ? 1 : 0;
   }
+  if (which == 3) return bha::full_prefix_tc_supports(full_args(dims, 0), bf16) ? 1 : 0;
   return 0;
 }
 
@@ -148,9 +161,12 @@ int bha_commit_block(const bha_dims* dims, const int32_t* cu_blk, const int32_t*
   return launch_status(bha::launch_commit_simt(a, bf16, static_cast<cudaStream_t>(stream)));
 }
 
+
 size_t bha_full_prefix_workspace_bytes(const bha_dims* dims, int64_t kv_capacity) {
-  if (check_dims(dims) != BHA_OK || kv_capacity < 0) return 0;
-  return 0;
+  if (check_dims(dims) != BHA_OK || kv_capacity < 0 || kv_capacity > INT32_MAX) return 0;
+  const bha::FullPrefixArgs a = full_args(dims, kv_capacity);
+  if (!bha::full_prefix_tc_supports(a, dims->act_dtype == BHA_BF16)) return 0;
+  return bha::full_prefix_tc_workspace(a);
 }
 
 int bha_full_prefix_attn(const bha_dims* dims, const int32_t* cu_blk, const int32_t* kv_len,
@@ -171,8 +187,10 @@ int bha_full_prefix_attn(const bha_dims* dims, const int32_t* cu_blk, const int3
   bha::FullPrefixArgs a{cu_blk, kv_len, Q, Kc, Vc, O, workspace, dev_err, kv_capacity,
                         dims->num_requests, dims->num_q_heads, dims->num_kv_heads,
                         dims->head_dim, dims->max_block, dims->total_tokens};
-  return launch_status(bha::launch_full_prefix_simt(a, dims->act_dtype == BHA_BF16,
-                                                    static_cast<cudaStream_t>(stream)));
+  const bool bf16 = dims->act_dtype == BHA_BF16;
+  if (bha::full_prefix_tc_supports(a, bf16))
+    return launch_status(bha::launch_full_prefix_tc(a, workspace, static_cast<cudaStream_t>(stream)));
+  return launch_status(bha::launch_full_prefix_simt(a, bf16, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -1,0 +1,461 @@
+// Tensor-core softmax teacher for sm_100a: exact attention of every active-block query over
+// its request's whole KV cache (committed prefix followed by the active block), unmasked.
+// bf16 activations, d = 128, four query heads per KV head, blocks of up to 32 tokens.
+//
+// Source: "Retrofitting Linear Attention into Diffusion Language Models", §2.2 (softmax
+// attention, exp(q.k/sqrt d)-weighted average of the visible values) and Appendix A (the
+// softmax kernel whose cost grows linearly with the prefix, kept here as the comparison
+// point for the block-hybrid layer).
+//
+// Work unit: (request r, KV head g, KV split s).  The 4 query heads x 32 block rows of (r, g)
+// form one 128-row MMA tile (as in the block-hybrid kernel); the unit sweeps its share of the
+// cache in 128-key tiles:
+//   S_i   = Q K_i^T              bf16 MMA into one of two TMEM score buffers (the next
+//                                tile's scores are computed while this tile's softmax runs)
+//   P_i   = 2^{S_i log2e/sqrt d - m_i}   online softmax, one thread per row, P in bf16
+//   D_i   = P_i V_i              bf16 MMA into one of two TMEM buffers
+//   O     = O 2^{m_{i-1} - m_i} + D_i    in registers
+// With one split the unit writes O / l; with several, it writes the unnormalised O, the
+// running max m (log2 units) and the sum l to the workspace and a combine kernel merges the
+// splits.  Keys at or past kv_len are masked by index and their V rows are cleared in
+// shared memory, so whatever the cache holds there (even non-finite bytes) has no effect.
+//
+// Roles (192 threads): warp 0 TMA producer (Q per unit, K/V tiles through a 2-stage ring),
+// warp 1 TMEM owner and MMA issuer, warps 2-5 softmax / accumulation / epilogue.  Every wait
+// is bounded; on expiry the CTA records BHA_ERR_TIMEOUT, drains, frees TMEM and returns.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_util.cuh"
+
+namespace bha {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kG = 4;
+constexpr int kBlk = 32;
+constexpr int kM = kG * kBlk;  // 128 query rows
+constexpr int kKT = 128;       // keys per tile
+constexpr int kStages = 2;
+constexpr int kThreads = 192;
+
+constexpr uint32_t kQBytes = kM * kD * 2;    // 32 KiB: [d half][128 rows][128 B]
+constexpr uint32_t kTileBytes = kKT * kD * 2;  // 32 KiB: [d half][128 keys][128 B]
+constexpr uint32_t kPBytes = kM * kKT * 2;   // 32 KiB: [key half][128 rows][128 B]
+
+constexpr uint32_t kColS = 0;    // two score buffers, 128 columns each
+constexpr uint32_t kColD = 256;  // two P V buffers, 128 columns each
+constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t kIdQK = tc::instr_desc(1, 0, 0, kM, kKT);
+constexpr uint32_t kIdPV = tc::instr_desc(1, 0, 1, kM, kD);
+
+struct __align__(1024) Smem {
+  uint8_t q[kQBytes];
+  uint8_t k[kStages][kTileBytes];
+  uint8_t v[kStages][kTileBytes];
+  uint8_t p[kPBytes];
+  uint64_t q_full, q_empty, kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], s_free[2], d_full[2], d_free[2], p_full, p_free, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory budget");
+
+struct Unit {
+  int r, g, s, lo, n, L, t0, nt;  // nt: number of 128-key tiles this split covers
+};
+
+__device__ __forceinline__ bool decode_unit(const TcFullParams& p, int u, bool report, Unit* x) {
+  x->s = u % p.nsplit;
+  const int pair = u / p.nsplit;
+  x->g = pair % p.Hkv;
+  x->r = pair / p.Hkv;
+  RowRange rr;
+  if (!request_rows(p.cu_blk, x->r, p.T, p.Bmax, p.dev_err, report, &rr)) return false;
+  if (rr.n == 0) return false;
+  const int L = p.kv_len[x->r];
+  if (L < 0 || L > p.cap) {
+    if (report) set_error(p.dev_err, BHA_ERR_INVALID);
+    return false;
+  }
+  x->lo = rr.lo;
+  x->n = rr.n;
+  x->L = L;
+  const int tiles = (L + kKT - 1) / kKT;
+  x->t0 = x->s * p.tiles_per_split;
+  x->nt = max(0, min(tiles, x->t0 + p.tiles_per_split) - x->t0);
+  return true;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) full_prefix_tc_kernel(const __grid_constant__ TcFullParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &sm.abort_flag;
+  const long long lim = p.wait_limit;
+  const int units = p.R * p.Hkv * p.nsplit;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&sm.q_full, 1);
+    tc::mbar_init(&sm.q_empty, 1);
+    for (int i = 0; i < kStages; ++i) {
+      tc::mbar_init(&sm.kv_full[i], 1);
+      tc::mbar_init(&sm.kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&sm.s_full[i], 1);
+      tc::mbar_init(&sm.s_free[i], 4);
+      tc::mbar_init(&sm.d_full[i], 1);
+      tc::mbar_init(&sm.d_free[i], 4);
+    }
+    tc::mbar_init(&sm.p_full, 4);
+    tc::mbar_init(&sm.p_free, 1);
+    tc::mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::prefetch_tensormap(&p.tm_q);
+    tc::prefetch_tensormap(&p.tm_k);
+    tc::prefetch_tensormap(&p.tm_v);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&sm.tmem_base, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int qk = 0, gt = 0;
+      int armed_q = -1, armed_kv[kStages] = {-1, -1};
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        Unit x;
+        if (!decode_unit(p, u, true, &x) || x.nt == 0) continue;
+        if (qk >= 1 && !tc::mbar_wait(&sm.q_empty, (qk - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        tc::mbar_arrive_expect_tx(&sm.q_full, kQBytes);
+        tc::tma_load_3d(sm.q, &p.tm_q, &sm.q_full, 0, kG * x.g, x.lo);
+        tc::tma_load_3d(sm.q + kQBytes / 2, &p.tm_q, &sm.q_full, 64, kG * x.g, x.lo);
+        armed_q = qk & 1;
+        ++qk;
+        const int row0 = (x.r * p.Hkv + x.g) * p.cap;
+        for (int i = 0; i < x.nt; ++i, ++gt) {
+          const int st = gt % kStages, j = gt / kStages;
+          if (j >= 1 && !tc::mbar_wait(&sm.kv_empty[st], (j - 1) & 1, abort_flag, lim)) { ok = false; break; }
+          tc::mbar_arrive_expect_tx(&sm.kv_full[st], 2 * kTileBytes);
+          const int key0 = row0 + (x.t0 + i) * kKT;
+          tc::tma_load_2d(sm.k[st], &p.tm_k, &sm.kv_full[st], 0, key0);
+          tc::tma_load_2d(sm.k[st] + kTileBytes / 2, &p.tm_k, &sm.kv_full[st], 64, key0);
+          tc::tma_load_2d(sm.v[st], &p.tm_v, &sm.kv_full[st], 0, key0);
+          tc::tma_load_2d(sm.v[st] + kTileBytes / 2, &p.tm_v, &sm.kv_full[st], 64, key0);
+          armed_kv[st] = j & 1;
+        }
+      }
+      volatile int never = 0;
+      if (armed_q >= 0) tc::mbar_wait(&sm.q_full, armed_q, &never, lim);
+      for (int st = 0; st < kStages; ++st)
+        if (armed_kv[st] >= 0) tc::mbar_wait(&sm.kv_full[st], armed_kv[st], &never, lim);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int qk = 0, gt = 0;
+      bool ok = true, issued = false;
+      auto issue_pv = [&](int tile) -> bool {
+        // P_tile V_tile into D buffer (tile & 1)
+        const int db = tile & 1, st = tile % kStages;
+        if (!tc::mbar_wait(&sm.p_full, tile & 1, abort_flag, lim)) return false;
+        if (tile >= 2 && !tc::mbar_wait(&sm.d_free[db], ((tile >> 1) - 1) & 1, abort_flag, lim)) return false;
+        tc::tc_fence_after();
+        const uint32_t pa = tc::smem_u32(sm.p), va = tc::smem_u32(sm.v[st]);
+#pragma unroll
+        for (int kk = 0; kk < kKT / 16; ++kk) {
+          const uint64_t a = tc::smem_desc(pa + (kk >> 2) * (kPBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
+          const uint64_t b = tc::smem_desc(va + kk * 2048, kTileBytes / 2, 1024, tc::kSwizzle128B);
+          tc::mma_bf16_ss(tbase + kColD + db * 128, a, b, kIdPV, kk > 0);
+        }
+        tc::mma_commit(&sm.d_full[db]);
+        tc::mma_commit(&sm.kv_empty[st]);
+        tc::mma_commit(&sm.p_free);
+        return true;
+      };
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        Unit x;
+        if (!decode_unit(p, u, false, &x) || x.nt == 0) continue;
+        if (!tc::mbar_wait(&sm.q_full, qk & 1, abort_flag, lim)) { ok = false; break; }
+        ++qk;
+        const uint32_t qa = tc::smem_u32(sm.q);
+        for (int i = 0; i < x.nt; ++i, ++gt) {
+          const int st = gt % kStages, sb = gt & 1;
+          if (!tc::mbar_wait(&sm.kv_full[st], (gt / kStages) & 1, abort_flag, lim)) { ok = false; break; }
+          if (gt >= 2 && !tc::mbar_wait(&sm.s_free[sb], ((gt >> 1) - 1) & 1, abort_flag, lim)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t ka = tc::smem_u32(sm.k[st]);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint64_t a = tc::smem_desc(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
+            const uint64_t b = tc::smem_desc(ka + (kk >> 2) * (kTileBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
+            tc::mma_bf16_ss(tbase + kColS + sb * 128, a, b, kIdQK, kk > 0);
+          }
+          tc::mma_commit(&sm.s_full[sb]);
+          if (i == x.nt - 1) tc::mma_commit(&sm.q_empty);
+          issued = true;
+          if (i >= 1 && !issue_pv(gt - 1)) { ok = false; break; }
+        }
+        if (!ok) break;
+        if (!issue_pv(gt - 1)) { ok = false; break; }
+      }
+      if (issued) {
+        volatile int never = 0;
+        tc::mma_commit(&sm.drain);
+        tc::mbar_wait(&sm.drain, 0, &never, lim);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / accumulation / epilogue
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;          // 4 t + head-in-group
+    const int t = row >> 2, hl = row & 3;
+    const int tid = threadIdx.x - 64;        // 0..127
+    const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
+    const float scale_log2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e)/sqrt(128)
+    int gt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      Unit x;
+      if (!decode_unit(p, u, false, &x)) continue;
+      float o[kD];
+#pragma unroll
+      for (int c = 0; c < kD; ++c) o[c] = 0.f;
+      float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
+      auto accumulate = [&](int tile, float alpha) -> bool {
+        const int db = tile & 1;
+        if (!tc::mbar_wait(&sm.d_full[db], (tile >> 1) & 1, abort_flag, lim)) return false;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kD / 32; ++c) {
+          float dv[32];
+          tc::tmem_ld32(tl + kColD + db * 128 + c * 32, dv);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha, dv[i]);
+        }
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&sm.d_free[db]);
+        return true;
+      };
+      for (int i = 0; i < x.nt; ++i, ++gt) {
+        const int sb = gt & 1, st = gt % kStages;
+        if (!tc::mbar_wait(&sm.s_full[sb], (gt >> 1) & 1, abort_flag, lim)) { ok = false; break; }
+        tc::tc_fence_after();
+        const int key0 = (x.t0 + i) * kKT;
+        const int valid_keys = min(kKT, x.L - key0);
+        const uint32_t scol = tl + kColS + sb * 128;
+        // pass 1: row max of this tile's scaled scores (keys at or past kv_len excluded)
+        float tmax = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < kKT / 32; ++c) {
+          float tmp[32];
+          tc::tmem_ld32(scol + c * 32, tmp);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (c * 32 + j < valid_keys) tmax = fmaxf(tmax, tmp[j] * scale_log2);
+        }
+        const float m_new = fmaxf(m, tmax);
+        const float alpha = (m_new == -INFINITY) ? 1.f : tc::ex2(m - m_new);
+        // P is free once the previous tile's P V has completed
+        if (gt >= 1 && !tc::mbar_wait(&sm.p_free, (gt - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        // pass 2: P = 2^{s - m_new} in bf16; keys [64 a, 64 a + 64) in atom a, 16-byte chunk c
+        // of a row at chunk c ^ (row % 8)
+        float psum = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < kKT / 32; ++c) {
+          float tmp[32];
+          tc::tmem_ld32(scol + c * 32, tmp);
+          tc::tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const bool v0 = c * 32 + j < valid_keys, v1 = c * 32 + j + 1 < valid_keys;
+            const float a0 = v0 ? tc::ex2(fmaf(tmp[j], scale_log2, -m_new)) : 0.f;
+            const float a1 = v1 ? tc::ex2(fmaf(tmp[j + 1], scale_log2, -m_new)) : 0.f;
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
+            psum += __low2float(b2) + __high2float(b2);
+            pk[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          uint8_t* prow = sm.p + (c >> 1) * (kPBytes / 2) + row * 128;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int ch = (c & 1) * 4 + q4;
+            *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
+                make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+          }
+        }
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&sm.s_free[sb]);
+        l = l * alpha + psum;
+        m = m_new;
+        if (valid_keys < kKT) {
+          // V rows past kv_len are cleared (the cache may hold anything there)
+          const int per_half = (kKT - valid_keys) * 8;
+          for (int q = tid; q < 2 * per_half; q += 128) {
+            const int hh = q / per_half, rem = q % per_half;
+            *reinterpret_cast<uint4*>(sm.v[st] + hh * (kTileBytes / 2) + (valid_keys + rem / 8) * 128 + (rem % 8) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+        }
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&sm.p_full);
+        if (i >= 1 && !accumulate(gt - 1, alpha_prev)) { ok = false; break; }
+        alpha_prev = alpha;
+      }
+      if (!ok) break;
+      if (x.nt > 0 && !accumulate(gt - 1, alpha_prev)) { ok = false; break; }
+      // epilogue
+      if (t < x.n) {
+        const size_t orow = (size_t)(x.lo + t) * p.Hq + kG * x.g + hl;
+        if (p.nsplit == 1) {
+          const float inv = l > 0.f ? 1.f / l : 0.f;
+          __nv_bfloat16* op = p.O + orow * kD;
+#pragma unroll
+          for (int c = 0; c < kD; c += 8)
+            *reinterpret_cast<uint4*>(op + c) =
+                make_uint4(pack_bf16(o[c] * inv, o[c + 1] * inv), pack_bf16(o[c + 2] * inv, o[c + 3] * inv),
+                           pack_bf16(o[c + 4] * inv, o[c + 5] * inv), pack_bf16(o[c + 6] * inv, o[c + 7] * inv));
+        } else {
+          const size_t prow = (size_t)x.s * p.T * p.Hq + orow;
+          float* op = p.opart + prow * kD;
+#pragma unroll
+          for (int c = 0; c < kD; c += 4) *reinterpret_cast<float4*>(op + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+          p.mpart[prow] = m;
+          p.lpart[prow] = l;
+        }
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);
+  if (threadIdx.x == 0 && sm.abort_flag) set_error(p.dev_err, BHA_ERR_TIMEOUT);
+}
+
+// Merges the splits of one (request, query head): O = sum_s 2^{m_s - m*} O_s / sum_s 2^{m_s - m*} l_s.
+__global__ void __launch_bounds__(128) combine_splits_kernel(const TcFullParams p) {
+  const int r = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
+  RowRange rr;
+  if (!request_rows(p.cu_blk, r, p.T, p.Bmax, p.dev_err, false, &rr)) return;
+  const int L = p.kv_len[r];
+  if (L < 0 || L > p.cap) return;
+  for (int i = 0; i < rr.n; ++i) {
+    const size_t orow = (size_t)(rr.lo + i) * p.Hq + h;
+    float mx = -INFINITY;
+    for (int s = 0; s < p.nsplit; ++s) mx = fmaxf(mx, p.mpart[(size_t)s * p.T * p.Hq + orow]);
+    float num = 0.f, den = 0.f;
+    if (mx != -INFINITY) {
+      for (int s = 0; s < p.nsplit; ++s) {
+        const size_t prow = (size_t)s * p.T * p.Hq + orow;
+        const float ms = p.mpart[prow];
+        if (ms == -INFINITY) continue;
+        const float w = tc::ex2(ms - mx);
+        num = fmaf(w, p.opart[prow * kD + d], num);
+        den = fmaf(w, p.lpart[prow], den);
+      }
+    }
+    p.O[orow * kD + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+  }
+}
+
+}  // namespace
+
+bool full_prefix_tc_supports(const FullPrefixArgs& a, bool act_bf16) {
+  return act_bf16 && a.d == kD && a.Hq == kG * a.Hkv && a.Bmax <= kBlk &&
+         (long long)a.R * a.Hkv * (a.kv_capacity + kKT) < (1ll << 31);
+}
+
+// Number of KV splits per (request, KV head): enough units to cover the SMs several times,
+// each split at least 4 tiles long.  Depends only on the call's dims and cache capacity.
+int full_prefix_splits(int R, int Hkv, int64_t cap) {
+  const long long pairs = (long long)R * Hkv;
+  const long long tiles = (cap + kKT - 1) / kKT;
+  if (pairs <= 0 || tiles <= 0) return 1;
+  long long want = (148 * 8 + pairs - 1) / pairs;
+  long long most = (tiles + 3) / 4;
+  long long s = want < most ? want : most;
+  if (s < 1) s = 1;
+  if (s > 64) s = 64;
+  return (int)s;
+}
+
+size_t full_prefix_tc_workspace(const FullPrefixArgs& a) {
+  const int ns = full_prefix_splits(a.R, a.Hkv, a.kv_capacity);
+  if (ns <= 1) return 0;
+  return (size_t)ns * a.T * a.Hq * (kD + 2) * sizeof(float);
+}
+
+cudaError_t launch_full_prefix_tc(const FullPrefixArgs& a, void* workspace, cudaStream_t st) {
+  TcFullParams p;
+  {
+    const uint64_t dims[3] = {kD, (uint64_t)a.Hq, (uint64_t)a.T};
+    const uint64_t strides[2] = {kD * 2, (uint64_t)a.Hq * kD * 2};
+    const uint32_t box[3] = {64, kG, kBlk};
+    if (!make_tensor_map(&p.tm_q, false, 3, a.Q, dims, strides, box, false)) return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[2] = {kD, (uint64_t)a.R * a.Hkv * a.kv_capacity};
+    const uint64_t strides[1] = {kD * 2};
+    const uint32_t box[2] = {64, kKT};
+    if (!make_tensor_map(&p.tm_k, false, 2, a.Kc, dims, strides, box, false)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&p.tm_v, false, 2, a.Vc, dims, strides, box, false)) return cudaErrorInvalidValue;
+  }
+  p.cu_blk = a.cu_blk;
+  p.kv_len = a.kv_len;
+  p.O = static_cast<__nv_bfloat16*>(a.O);
+  p.dev_err = a.dev_err;
+  p.R = a.R;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.T = a.T;
+  p.Bmax = a.Bmax;
+  p.cap = (int)a.kv_capacity;
+  p.nsplit = full_prefix_splits(a.R, a.Hkv, a.kv_capacity);
+  const int tiles_cap = (int)((a.kv_capacity + kKT - 1) / kKT);
+  p.tiles_per_split = (tiles_cap + p.nsplit - 1) / p.nsplit;
+  if (p.tiles_per_split < 1) p.tiles_per_split = 1;
+  p.wait_limit = 2000000000ll;
+  if (p.nsplit > 1) {
+    float* ws = static_cast<float*>(workspace);
+    const size_t rows = (size_t)p.nsplit * a.T * a.Hq;
+    p.opart = ws;
+    p.mpart = ws + rows * kD;
+    p.lpart = p.mpart + rows;
+  } else {
+    p.opart = p.mpart = p.lpart = nullptr;
+  }
+  const int units = a.R * a.Hkv * p.nsplit;
+  int nsm = device_sm_count();
+  if (nsm <= 0) return cudaErrorInvalidDevice;
+  const int grid = units < nsm ? units : nsm;
+  const size_t smem = sizeof(Smem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(full_prefix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  full_prefix_tc_kernel<<<grid, kThreads, smem, st>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.nsplit == 1) return e;
+  combine_splits_kernel<<<dim3(a.R, a.Hq), 128, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace bha

@@ -75,6 +75,20 @@ struct TcCommitParams {
   long long wait_limit;
 };
 
+// Parameters of the tensor-core softmax-teacher kernel (full_prefix_tc.cu).
+struct TcFullParams {
+  CUtensorMap tm_q, tm_k, tm_v;
+  const int32_t* cu_blk;
+  const int32_t* kv_len;
+  __nv_bfloat16* O;
+  float* opart;  // [nsplit][T * Hq][d] unnormalised partial outputs
+  float* mpart;  // [nsplit][T * Hq] running max (log2 units)
+  float* lpart;  // [nsplit][T * Hq] softmax sums
+  int32_t* dev_err;
+  int R, Hq, Hkv, T, Bmax, cap, nsplit, tiles_per_split;
+  long long wait_limit;
+};
+
 // host helpers shared by the tensor-core launchers (hybrid_tc.cu)
 bool make_tensor_map(CUtensorMap* m, bool f32, int rank, const void* base, const uint64_t* dims,
                      const uint64_t* strides_bytes, const uint32_t* box, bool swizzle_atom32);
@@ -85,6 +99,10 @@ bool hybrid_tc_supports(const HybridArgs& a, bool act_bf16);
 cudaError_t launch_hybrid_tc(const HybridArgs& a, cudaStream_t st);
 bool commit_tc_supports(const CommitArgs& a, bool act_bf16);
 cudaError_t launch_commit_tc(const CommitArgs& a, cudaStream_t st);
+bool full_prefix_tc_supports(const FullPrefixArgs& a, bool act_bf16);
+int full_prefix_splits(int R, int Hkv, int64_t cap);
+size_t full_prefix_tc_workspace(const FullPrefixArgs& a);
+cudaError_t launch_full_prefix_tc(const FullPrefixArgs& a, void* workspace, cudaStream_t st);
 
 // generic CUDA-core kernels (simt.cu)
 bool simt_supports(int d, int F, int Bmax);

@@ -269,6 +269,7 @@ def test_tensor_core_path_is_taken_for_the_serving_shape():
     assert bha.kernel_variant(d32, 1) == 0   # fp32 activations take the fp32 CUDA-core path
     assert bha.kernel_variant(d, 2) == 1     # block commit on tensor cores
     assert bha.kernel_variant(d32, 2) == 0
+    assert bha.kernel_variant(d, 3) == 1     # softmax teacher on tensor cores
 
 
 def test_linear_branch_dominant_states():
@@ -306,3 +307,49 @@ def test_zero_weight_closed_form_full_size():
     den = a.sum(-1).transpose(0, 2, 1)[..., None] + 2.0 * P / Fh
     want = (num / den).reshape(4096, 16, 128)
     assert_close(O, want, TOL_BF16, "O (closed form)")
+
+
+@pytest.mark.parametrize("poison", [False, True])
+def test_full_prefix_teacher_split_kv(poison):
+    """Long caches take the split-KV path (partials in the workspace, then a combine).  Cache
+    rows past kv_len may hold anything: with poison=True they are NaN and must not matter."""
+    R, Hq, Hkv, d, cap = 3, 8, 2, 128, 2000
+    kv_len = np.array([2000, 130, 0], dtype=np.int32)
+    lens = np.array([32, 17, 5])
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    rng = np.random.default_rng(21)
+    Q = inputs.bf16_round(rng.standard_normal((cu[-1], Hq, d)).astype(np.float32))
+    Kc = inputs.bf16_round(rng.standard_normal((R, Hkv, cap, d)).astype(np.float32))
+    Vc = inputs.bf16_round(rng.standard_normal((R, Hkv, cap, d)).astype(np.float32))
+    tK, tV = dev(Kc, torch.bfloat16), dev(Vc, torch.bfloat16)
+    if poison:
+        for r in range(R):
+            tK[r, :, kv_len[r]:] = float("nan")
+            tV[r, :, kv_len[r]:] = float("nan")
+    assert bha.full_prefix_workspace_bytes(R, Hq, Hkv, d, 32, int(cu[-1]), cap) > 0
+    O = bha.full_prefix_attn(torch.tensor(cu, device="cuda"), torch.tensor(kv_len, device="cuda"),
+                             dev(Q, torch.bfloat16), tK, tV, max_block=32)
+    torch.cuda.synchronize()
+    want = ref.full_prefix_attn(cu, kv_len, Q, Kc, Vc)
+    assert_close(host64(O), want, TOL_BF16, "O")
+
+
+def test_full_prefix_teacher_serving_size_sampled():
+    """64 requests, 16 query / 4 KV heads, 2048-token prefixes plus the 32-token block; every
+    output row of 6 sampled requests checked against the oracle."""
+    R, Hq, Hkv, d, P = 64, 16, 4, 128, 2048
+    L = P + 32
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    Kc = torch.randn((R, Hkv, L, d), generator=g, device="cuda").to(torch.bfloat16)
+    Vc = torch.randn((R, Hkv, L, d), generator=g, device="cuda").to(torch.bfloat16)
+    Q = torch.randn((R * 32, Hq, d), generator=g, device="cuda").to(torch.bfloat16)
+    cu = torch.arange(0, (R + 1) * 32, 32, dtype=torch.int32, device="cuda")
+    kv_len = torch.full((R,), L, dtype=torch.int32, device="cuda")
+    O = host64(bha.full_prefix_attn(cu, kv_len, Q, Kc, Vc, max_block=32))
+    reqs = np.random.default_rng(2).choice(R, 6, replace=False)
+    Qh, Kh, Vh = host64(Q), host64(Kc), host64(Vc)
+    for r in reqs:
+        sl = slice(32 * r, 32 * r + 32)
+        want = ref.full_prefix_attn([0, 32], [L], Qh[sl], Kh[r:r + 1], Vh[r:r + 1])
+        assert_close(O[sl], want, TOL_BF16, f"O[{r}]")
