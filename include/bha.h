@@ -117,6 +117,30 @@ int bha_full_prefix_attn(const bha_dims* dims, const int32_t* cu_blk, const int3
 /* Scratch bytes bha_full_prefix_attn needs for these dims and cache capacity. */
 size_t bha_full_prefix_workspace_bytes(const bha_dims* dims, int64_t kv_capacity);
 
+/* Size of the fixed scratch array behind bha_full_prefix_attn_noalloc (16 MiB). */
+#define BHA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* bha_full_prefix_attn without the caller-provided workspace.  The paper has no counterpart:
+ * this exists for callers that cannot allocate device memory on the call path -- for
+ * example a serving engine that reserves its whole memory budget up front and forbids
+ * cudaMalloc inside the decode loop, or a plugin whose host owns all allocation.
+ *   Arguments, layouts, results and dev_err behave exactly as in bha_full_prefix_attn.
+ *   The split partials go to a file-scope device array of BHA_NOALLOC_SCRATCH_BYTES that
+ *   every GPU loading the library holds until the process exits.  The call allocates
+ *   nothing (no cudaMalloc / cudaFree and no allocating library routine).
+ *   Returns BHA_ERR_UNSUPPORTED, launching nothing, when the call would need more scratch
+ *   than that (bha_full_prefix_workspace_bytes(dims, kv_capacity) >
+ *   BHA_NOALLOC_SCRATCH_BYTES).
+ *   The first call on each device, with that device current, looks up the array's device
+ *   address (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   All calls share the one array and it keeps the last call's contents (nothing in it has
+ *   to start at zero), so calls whose kernels may overlap on the GPU -- different streams,
+ *   or different host threads -- race on it and must be serialised by the caller. */
+int bha_full_prefix_attn_noalloc(const bha_dims* dims, const int32_t* cu_blk,
+                                 const int32_t* kv_len, const void* Q, const void* Kc,
+                                 const void* Vc, int64_t kv_capacity, void* O, int32_t* dev_err,
+                                 void* stream);
+
 /* Static description of a status code. */
 const char* bha_status_string(int status);
 

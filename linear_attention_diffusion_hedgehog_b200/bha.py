@@ -53,6 +53,8 @@ _SIGS = {
     "bha_full_prefix_attn": (ctypes.c_int, [ctypes.POINTER(Dims), _P, _P, _P, _P, _P,
                                             ctypes.c_int64, _P, _P, ctypes.c_size_t, _P, _P]),
     "bha_full_prefix_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int64]),
+    "bha_full_prefix_attn_noalloc": (ctypes.c_int, [ctypes.POINTER(Dims), _P, _P, _P, _P, _P,
+                                                    ctypes.c_int64, _P, _P, _P]),
     "bha_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bha_kernel_variant": (ctypes.c_int, [ctypes.POINTER(Dims), _I32]),
     "bha_version": (ctypes.c_int, []),
@@ -249,4 +251,34 @@ def full_prefix_attn(cu_blk, kv_len, Q, Kc, Vc, *, max_block, workspace=None, ou
                                     _ptr(Kc), _ptr(Vc), cap, _ptr(out), _ptr(workspace), wbytes,
                                     _ptr(dev_err), _stream(Q.device, stream))
     _check(st, "bha_full_prefix_attn")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def full_prefix_attn_noalloc(cu_blk, kv_len, Q, Kc, Vc, *, max_block, out=None, dev_err=None,
+                             stream=None):
+    """Softmax teacher without a caller workspace: the split partials use the library's fixed
+    device scratch array (shared by every call; concurrent calls must be serialised)."""
+    _cuda(Q, "Q", ndim=3)
+    dt = Q.dtype
+    _cuda(Kc, "Kc", dtype=dt, ndim=4)
+    _cuda(Vc, "Vc", dtype=dt, ndim=4)
+    _cuda(cu_blk, "cu_blk", dtype=torch.int32, ndim=1)
+    _cuda(kv_len, "kv_len", dtype=torch.int32, ndim=1)
+    T, Hq, d = Q.shape
+    R, Hkv, cap, dk = Kc.shape
+    _need(dk == d and tuple(Vc.shape) == tuple(Kc.shape), "Kc/Vc must be [R, Hkv, capacity, d]")
+    _need(cu_blk.shape[0] == R + 1 and kv_len.shape[0] == R, "cu_blk [R+1], kv_len [R]")
+    if out is None:
+        out = torch.empty_like(Q)
+    _cuda(out, "out", dtype=dt, ndim=3)
+    if dev_err is not None:
+        _cuda(dev_err, "dev_err", dtype=torch.int32)
+    dims = make_dims(R, Hq, Hkv, d, 2, max_block, T, 0, dt)
+    st = lib().bha_full_prefix_attn_noalloc(ctypes.byref(dims), _ptr(cu_blk), _ptr(kv_len),
+                                            _ptr(Q), _ptr(Kc), _ptr(Vc), cap, _ptr(out),
+                                            _ptr(dev_err), _stream(Q.device, stream))
+    _check(st, "bha_full_prefix_attn_noalloc")
     return out
