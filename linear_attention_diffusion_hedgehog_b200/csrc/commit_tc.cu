@@ -395,14 +395,14 @@ cudaError_t launch_commit_tc(const CommitArgs& a, cudaStream_t st) {
     const uint64_t dims[3] = {kD, (uint64_t)a.Hkv, T};
     const uint64_t strides[2] = {kD * 2, (uint64_t)a.Hkv * kD * 2};
     const uint32_t box[3] = {64, 1, kBlk};
-    if (!make_tensor_map(&p.tm_k, false, 3, a.K, dims, strides, box, false)) return cudaErrorInvalidValue;
-    if (!make_tensor_map(&p.tm_v, false, 3, a.V, dims, strides, box, false)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&p.tm_k, false, 3, a.K, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&p.tm_v, false, 3, a.V, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
   }
   {
     const uint64_t dims[2] = {kFh, (uint64_t)a.Hkv * kD};
     const uint64_t strides[1] = {kFh * 2};
     const uint32_t box[2] = {64, kD};
-    if (!make_tensor_map(&p.tm_w, false, 2, a.W, dims, strides, box, false)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&p.tm_w, false, 2, a.W, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
   }
   p.cu_blk = a.cu_blk;
   p.state_slot = a.state_slot;

@@ -411,14 +411,14 @@ cudaError_t launch_full_prefix_tc(const FullPrefixArgs& a, void* workspace, cuda
     const uint64_t dims[3] = {kD, (uint64_t)a.Hq, (uint64_t)a.T};
     const uint64_t strides[2] = {kD * 2, (uint64_t)a.Hq * kD * 2};
     const uint32_t box[3] = {64, kG, kBlk};
-    if (!make_tensor_map(&p.tm_q, false, 3, a.Q, dims, strides, box, false)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&p.tm_q, false, 3, a.Q, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
   }
   {
     const uint64_t dims[2] = {kD, (uint64_t)a.R * a.Hkv * a.kv_capacity};
     const uint64_t strides[1] = {kD * 2};
     const uint32_t box[2] = {64, kKT};
-    if (!make_tensor_map(&p.tm_k, false, 2, a.Kc, dims, strides, box, false)) return cudaErrorInvalidValue;
-    if (!make_tensor_map(&p.tm_v, false, 2, a.Vc, dims, strides, box, false)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&p.tm_k, false, 2, a.Kc, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&p.tm_v, false, 2, a.Vc, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
   }
   p.cu_blk = a.cu_blk;
   p.kv_len = a.kv_len;

@@ -52,7 +52,7 @@ struct FullPrefixArgs {
 // Parameters of the tensor-core decode-step kernel (hybrid_tc.cu); the tensor maps describe
 // Q, K, V, W and S for the Tensor Memory Accelerator.
 struct TcHybridParams {
-  CUtensorMap tm_q, tm_k, tm_v, tm_w, tm_s;
+  CUtensorMap tm_q, tm_k, tm_v, tm_w, tm_s, tm_o;
   const int32_t* cu_blk;
   const int32_t* state_slot;
   const float* Z;
@@ -89,9 +89,10 @@ struct TcFullParams {
   long long wait_limit;
 };
 
-// host helpers shared by the tensor-core launchers (hybrid_tc.cu)
+// host helpers shared by the tensor-core launchers (tc_host.cu)
+enum TmaSwizzle { kTma128B, kTma128BAtom32, kTmaNone };
 bool make_tensor_map(CUtensorMap* m, bool f32, int rank, const void* base, const uint64_t* dims,
-                     const uint64_t* strides_bytes, const uint32_t* box, bool swizzle_atom32);
+                     const uint64_t* strides_bytes, const uint32_t* box, TmaSwizzle swizzle);
 int device_sm_count();
 
 // tensor-core kernels
