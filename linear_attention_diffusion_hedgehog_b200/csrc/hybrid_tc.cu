@@ -57,7 +57,7 @@ constexpr int kBlk = 32;
 constexpr int kM = kG * kBlk;  // 128 tile rows
 constexpr int kChunk = 32;         // F rows of S per chunk = one group of 32 e values
 constexpr int kGroups = kFh / kChunk;  // groups of 32 e values per half
-constexpr int kStages = 3;         // S ring: each stage holds group g of both halves
+constexpr int kStages = 4;         // S ring: each stage holds group g of both halves
 constexpr int kThreads = 320;
 
 constexpr uint32_t kQBytes = kM * kD * 2;      // 32 KiB
@@ -66,7 +66,6 @@ constexpr uint32_t kZBytes = kF * 4;           // 1 KiB
 constexpr uint32_t kWBytes = kD * kFh * 2;     // 32 KiB
 constexpr uint32_t kSBytes = kChunk * kD * 4;  // 16 KiB fp32: [d quarter][32 rows][128 B]
 constexpr uint32_t kPBytes = kM * 64;          // 8 KiB (64-byte rows, 64-byte swizzle)
-constexpr uint32_t kOBytes = 8 * kG * 128;     // 4 KiB: one warp's 8 tokens x 4 heads x 64 columns
 
 // TMEM columns
 constexpr uint32_t kColU = 0;      // u = Q W_g, then e+ in place
@@ -88,11 +87,9 @@ struct __align__(1024) Smem {
                                    // 32-byte-atom swizzle
   uint8_t k[kKBytes];           // [d half][32 rows][128 B]
   uint8_t v[kKBytes];
-  uint8_t p[kPBytes];           // P: [128 rows][64 B], 64-byte swizzle
-  uint8_t o[8][kOBytes];        // per feature-map warp: output staging, 128-byte swizzle
+  uint8_t p[kPBytes];           // P: [128 rows][64 B], 64-byte swizzle; then output staging
   float z[2][kF];
-  float red[2][kM];             // per-row denominator parts
-  float scl[2][kM];             // per-row epilogue factors c+ and c-
+  float xch[7][2][kM];          // per-row values the two warps of a lane quarter exchange
   uint64_t qk_full, qk_empty, v_full, v_empty, v_ready, z_full[2], z_empty[2];
   uint64_t s_full[kStages], s_empty[kStages];
   uint64_t e_ready[kGroups], p_ready;
@@ -101,6 +98,7 @@ struct __align__(1024) Smem {
   int abort_flag;
 };
 static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory budget of one CTA per SM");
+static_assert(kStages <= kGroups, "V is loaded ahead of the S pair that reuses the first stage");
 
 struct Unit {
   int r, g, lo, n, slot;
@@ -108,6 +106,10 @@ struct Unit {
 
 // Decodes unit u and validates it; every role calls this with the same arguments and so
 // skips the same units.
+// Order in which the S pairs are loaded and contracted: warps 2-5 produce groups 0 and 1
+// while warps 6-9 produce groups 2 and 3, so groups 0 and 2 become ready first.
+__device__ __forceinline__ int group_at(int i) { return (i & 1) * 2 + (i >> 1); }
+
 __device__ __forceinline__ bool decode_unit(const TcHybridParams& p, int u, bool report, Unit* x) {
   x->g = u % p.Hkv;
   x->r = u / p.Hkv;
@@ -148,12 +150,12 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
       tc::mbar_init(&sm.z_full[i], 1);
       tc::mbar_init(&sm.z_empty[i], 8);
     }
-    for (int j = 0; j < kGroups; ++j) tc::mbar_init(&sm.e_ready[j], 8);
+    for (int j = 0; j < kGroups; ++j) tc::mbar_init(&sm.e_ready[j], 4);  // the 4 warps owning group j
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&sm.s_full[i], 1);
       tc::mbar_init(&sm.s_empty[i], 1);
     }
-    tc::mbar_init(&sm.p_ready, 4);
+    tc::mbar_init(&sm.p_ready, 8);
     tc::mbar_init(&sm.w_full, 1);
     tc::mbar_init(&sm.u_full, 1);
     tc::mbar_init(&sm.acc_full, 1);
@@ -215,7 +217,17 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
         tc::bulk_load(sm.z[zb], p.Z + ((size_t)x.slot * p.Hkv + x.g) * kF, kZBytes, &sm.z_full[zb]);
         armed_z[zb] = zj & 1;
         const int srow0 = (x.slot * p.Hkv + x.g) * kF;
-        for (int grp = 0; grp < kGroups; ++grp, ++q) {
+        for (int i = 0; i < kGroups; ++i, ++q) {
+          const int grp = group_at(i);
+          if (i == kStages - 1) {
+            // V (read by the unit's P V) goes ahead of the last S pair, which waits for the
+            // previous unit's last pair to be consumed, so that it lands before it is needed
+            if (k >= 1 && !tc::mbar_wait(&sm.v_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+            tc::mbar_arrive_expect_tx(&sm.v_full, kKBytes);
+            tc::tma_load_3d(sm.v, &p.tm_v, &sm.v_full, 0, x.g, x.lo);
+            tc::tma_load_3d(sm.v + kKBytes / 2, &p.tm_v, &sm.v_full, 64, x.g, x.lo);
+            armed_v = k & 1;
+          }
           const int st = q % kStages, j = q / kStages;
           if (j >= 1 && !tc::mbar_wait(&sm.s_empty[st], (j - 1) & 1, abort_flag, lim)) { ok = false; break; }
           tc::mbar_arrive_expect_tx(&sm.s_full[st], 2 * kSBytes);
@@ -227,13 +239,6 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
                               srow0 + hf * kFh + grp * kChunk);
           armed_s[st] = j & 1;
         }
-        if (!ok) break;
-        // V is read last, by the unit's P V
-        if (k >= 1 && !tc::mbar_wait(&sm.v_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
-        tc::mbar_arrive_expect_tx(&sm.v_full, kKBytes);
-        tc::tma_load_3d(sm.v, &p.tm_v, &sm.v_full, 0, x.g, x.lo);
-        tc::tma_load_3d(sm.v + kKBytes / 2, &p.tm_v, &sm.v_full, 64, x.g, x.lo);
-        armed_v = k & 1;
       }
       // Drain: every copy this thread started has landed before the CTA can exit.
       volatile int never = 0;
@@ -260,7 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
           g_res = x.g;
         }
         // u and the scores overwrite e+ and the top of e-, which the previous unit's MMAs read
-        if (k >= 1 && !tc::mbar_wait(&sm.acc_full, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        // as their A operand: MMAs issued by one thread execute in issue order, so these are
+        // issued right behind them without waiting for them to complete
         if (!tc::mbar_wait(&sm.qk_full, k & 1, abort_flag, lim)) { ok = false; break; }
         tc::tc_fence_after();
         const uint32_t qa = tc::smem_u32(sm.q);
@@ -285,25 +291,24 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
         if (k >= 1 && !tc::mbar_wait(&sm.acc_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
         // A+ += e+ S+ and A- += e- S-, group by group as the feature-map warps release them
         // (one wait per group for both halves keeps this thread's per-MMA overhead low)
-        for (int grp = 0; grp < kGroups; ++grp, ++q) {
+        for (int i = 0; i < kGroups; ++i, ++q) {
+          const int grp = group_at(i);
           if (!tc::mbar_wait(&sm.e_ready[grp], k & 1, abort_flag, lim)) { ok = false; break; }
           const int st = q % kStages;
           if (!tc::mbar_wait(&sm.s_full[st], (q / kStages) & 1, abort_flag, lim)) { ok = false; break; }
           tc::tc_fence_after();
-          const uint32_t sa = tc::smem_u32(sm.s[st][0]);
-          const uint32_t ep = tbase + kColU + grp * 32, em = tbase + kColEm + grp * 32;
           // MN-major tf32 B: 128-byte swizzle with 32-byte atoms, 4-row K groups (SBO 512 B),
-          // d quarters 4 KiB apart (LBO); K steps of 8 rows are 1 KiB apart
+          // d quarters 4 KiB apart (LBO); K steps of 8 rows are 1 KiB apart, i.e. 64 in the
+          // descriptor's 16-byte address units
+          const uint64_t bp = tc::smem_desc(tc::smem_u32(sm.s[st][0]), kSBytes / 4, 512, tc::kSwizzle128BBase32B);
+          const uint64_t bm = bp + (kSBytes >> 4);
+          const uint32_t ep = tbase + kColU + grp * 32, em = tbase + kColEm + grp * 32;
 #pragma unroll
           for (int kk = 0; kk < kChunk / 8; ++kk)
-            tc::mma_tf32_ts(tbase + kColAp, ep + kk * 8,
-                            tc::smem_desc(sa + kk * 1024, kSBytes / 4, 512, tc::kSwizzle128BBase32B), kIdES,
-                            (grp > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_tf32_ts(tbase + kColAp, ep + kk * 8, bp + (uint64_t)(kk * 64), kIdES, (i > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < kChunk / 8; ++kk)
-            tc::mma_tf32_ts(tbase + kColAm, em + kk * 8,
-                            tc::smem_desc(sa + kSBytes + kk * 1024, kSBytes / 4, 512, tc::kSwizzle128BBase32B),
-                            kIdES, (grp > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_tf32_ts(tbase + kColAm, em + kk * 8, bm + (uint64_t)(kk * 64), kIdES, (i > 0 || kk > 0) ? 1u : 0u);
           tc::mma_commit(&sm.s_empty[st]);
         }
         if (!ok) break;
@@ -330,84 +335,106 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
     }
   } else {
     // ------------------------------------------------------------ feature map / epilogue
+    // The two warps of a TMEM lane quarter share its 32 tile rows: warp part 0 (warps 2-5)
+    // takes feature groups 0 and 1 of u, part 1 (warps 6-9) groups 2 and 3; each computes both
+    // e+ and e- of its groups from one read of u, half of the block keys of P, and half of
+    // the output columns.  They exchange per-row values through shared memory at three pair
+    // barriers per unit (X1: max/min of u, X2: partial sums, X3: partial P sum).
     const int sw = warp - 2;           // 0..7
-    const int half = sw >> 2;          // 0: e+ half, 1: e- half
-    const float sgn = half ? -1.f : 1.f;
+    const int part = sw >> 2;          // 0: groups 0-1, keys 0-15, columns 0-63; 1: the rest
     const int wq = warp & 3;           // TMEM lane quarter this warp may access
     const int row = wq * 32 + lane;    // tile row = 4 t + head-in-group
     const int hl = row & 3;
     const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
+    const uint32_t pair_bar = 2 + wq;
     const float scale_log2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
     const float log2e = 1.4426950408889634f;
+    const int g0 = part * 2;           // this warp's first feature group
+    float* mine = &sm.xch[0][part][row];
+    const float* theirs = &sm.xch[0][part ^ 1][row];
+    constexpr int kX = 2 * kM;         // stride between exchange slots
     int ucur = blockIdx.x;
     Unit x{};
-    // A failed wait does not leave the loop at once: these 256 threads meet at named barriers,
-    // so every one of them finishes the unit's barriers and they leave together, decided by
-    // the reducing barrier below.  Work done after a failed wait is discarded.
+    // A failed wait does not leave the loop at once: the two warps of a pair meet at named
+    // barriers, so both finish the unit's barriers and leave together, decided by the
+    // reducing barrier at its end.  Work done after a failed wait is discarded.
     bool good = true;
     for (int k = 0; next_unit(p, units, &ucur, false, &x); ++k) {
       good = tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim) && good;
       good = tc::mbar_wait(&sm.z_full[k & 1], (k >> 1) & 1, abort_flag, lim) && good;
       tc::tc_fence_after();
 
+      float sv[32], u0[32], u1[32];
+      tc::tmem_ld32(tl + kColS, sv);
+      tc::tmem_ld32(tl + kColU + g0 * 32, u0);
+      tc::tmem_ld32(tl + kColU + g0 * 32 + 32, u1);
+      tc::tmem_wait_ld();
+
       // block softmax over the x.n keys of this request (bidirectional, no mask):
-      // a_j = w 2^{s_j log2e / sqrt d - m}, kept in fp32 until P's scale is known
-      float av[32];
+      // a_j = w 2^{s_j log2e / sqrt d - m}; this warp keeps its 16 keys in fp32 until P's
+      // scale is known
+      float av[16];
       float m2;
       {
-        float sv[32];
-        tc::tmem_ld32(tl + kColS, sv);
-        tc::tmem_wait_ld();
         float mraw = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           if (j < x.n) mraw = fmaxf(mraw, sv[j]);
         // m in log2 units, kept in [-6 log2 e, 90] so that 2^{-m} is finite and not tiny
         m2 = fminf(fmaxf(mraw * scale_log2, -6.f * log2e), 90.f);
-        const float wgt = (half == 0 && p.alpha) ? 1.f / (1.f + expf(-p.alpha[kG * x.g + hl])) : 1.f;
+        const float wgt = p.alpha ? 1.f / (1.f + expf(-p.alpha[kG * x.g + hl])) : 1.f;
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          av[j] = (half == 0 && j < x.n) ? wgt * tc::ex2(fmaf(sv[j], scale_log2, -m2)) : 0.f;
+        for (int j = 0; j < 16; ++j) {
+          const int jj = part * 16 + j;
+          const float s_j = part ? sv[16 + j] : sv[j];
+          av[j] = jj < x.n ? wgt * tc::ex2(fmaf(s_j, scale_log2, -m2)) : 0.f;
+        }
       }
       const float em = tc::ex2(-m2);
-      // every thread has read its scores before the e- half overwrites them
-      tc::tc_fence_before();
-      tc::named_barrier_sync(1, 256);
-      tc::tc_fence_after();
 
-      // this half of e, group by group (32 values), each group released to the MMA as soon
-      // as the four warps of this half have written it.  e+ overwrites u in place: the two
-      // warps that share a TMEM lane quarter meet at a barrier after reading each group of u.
-      float ext = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < kGroups; ++c) {
-        float uv[32];
-        tc::tmem_ld32(tl + kColU + c * 32, uv);
-        tc::tmem_wait_ld();
+      // X1: max and min of u over the row's 128 features
+      float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ext = fmaxf(ext, sgn * uv[i]);
+      for (int i = 0; i < 32; ++i) {
+        mx = fmaxf(mx, fmaxf(u0[i], u1[i]));
+        mn = fminf(mn, fminf(u0[i], u1[i]));
       }
-      const float ext2 = ext * log2e;
-      const float slog2e = sgn * log2e;
-      float esum = 0.f, zsum = 0.f;
-      const float* zb = sm.z[k & 1] + half * kFh;
-      const uint32_t e_col = half ? kColEm : kColU;
-#pragma unroll 1
-      for (int c = 0; c < kGroups; ++c) {
-        float uv[32];
-        tc::tmem_ld32(tl + kColU + c * 32, uv);
-        tc::tmem_wait_ld();
-        tc::tc_fence_before();
-        tc::named_barrier_sync(2 + wq, 64);  // both halves have read this group of u
-        tc::tc_fence_after();
+      mine[0 * kX] = mx;
+      mine[1 * kX] = mn;
+      // (both warps have also read the scores, which e- group 3 overwrites, by this barrier)
+      tc::tc_fence_before();
+      tc::named_barrier_sync(pair_bar, 64);
+      tc::tc_fence_after();
+      mx = fmaxf(mx, theirs[0 * kX]);
+      mn = fminf(mn, theirs[1 * kX]);
+
+      // e+_f = 2^{(u_f - max u) log2e} over u in place, e-_f = 2^{(min u - u_f) log2e}, group by
+      // group, each released to the MMA as soon as the four warps owning it have written it
+      const float bpl = mx * log2e, bml = mn * log2e;
+      const float* zk = sm.z[k & 1];
+      float esp = 0.f, esm = 0.f, zsp = 0.f, zsm = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float e = tc::ex2(fmaf(uv[i], slog2e, -ext2));
-          esum += e;
-          zsum = fmaf(e, zb[c * 32 + i], zsum);
-          uv[i] = e;
+      for (int gi = 0; gi < 2; ++gi) {
+        float(&uu)[32] = gi ? u1 : u0;
+        const int c = g0 + gi;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float ep[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a = uu[16 * h + i] * log2e;
+            const float e1 = tc::ex2(a - bpl);
+            const float e2 = tc::ex2(bml - a);
+            esp += e1;
+            esm += e2;
+            zsp = fmaf(e1, zk[c * 32 + 16 * h + i], zsp);
+            zsm = fmaf(e2, zk[kFh + c * 32 + 16 * h + i], zsm);
+            ep[i] = e1;
+            uu[16 * h + i] = e2;
+          }
+          tc::tmem_st16(tl + kColU + c * 32 + 16 * h, ep);
         }
-        tc::tmem_st32(tl + e_col + c * 32, uv);
+        tc::tmem_st32(tl + kColEm + c * 32, uu);
         tc::tmem_wait_st();
         tc::tc_fence_before();
         __syncwarp();
@@ -415,7 +442,19 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
       }
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.z_empty[k & 1]);
-      if (half == 0) {
+
+      // X2: the partial sums
+      mine[2 * kX] = esp;
+      mine[3 * kX] = esm;
+      mine[4 * kX] = zsp;
+      mine[5 * kX] = zsm;
+      tc::named_barrier_sync(pair_bar, 64);
+      esp += theirs[2 * kX];
+      esm += theirs[3 * kX];
+      zsp += theirs[4 * kX];
+      zsm += theirs[5 * kX];
+
+      if (part == 0) {
         // V of this unit: rows past a short block belong to another request; clear them
         good = tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim) && good;
         if (x.n < kBlk) {
@@ -431,93 +470,85 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
         if (lane == 0) tc::mbar_arrive(&sm.v_ready);
       }
 
-      // P (bf16, scaled by kappa = sum e+ / e^{-m}), the denominator parts and the epilogue
-      // factors c+/- = e^{-m} / sum e+/-
-      if (half == 0) {
-        const float kappa = esum / em;
-        uint32_t packed[16];
-        float psum = 0.f;
+      // P (bf16, scaled by kappa = sum e+ / e^{-m}): this warp's 16 keys, two 16-byte chunks of
+      // the row's 64 bytes (chunk c stored at chunk c ^ ((row / 2) % 4), the 64-byte swizzle)
+      const float kappa = esp / em;
+      float psum = 0.f;
+      {
+        uint32_t packed[8];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
+        for (int j = 0; j < 16; j += 2) {
           const __nv_bfloat162 b2 = __floats2bfloat162_rn(av[j] * kappa, av[j + 1] * kappa);
           psum += __low2float(b2) + __high2float(b2);
           packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
         }
-        // P row: 64 bytes, 16-byte chunk c at chunk c ^ ((row / 2) % 4) (64-byte swizzle)
         uint8_t* prow = sm.p + row * 64;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ ((row >> 1) & 3)) << 4)) =
-              make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&sm.p_ready);
-        // the denominator sums the same rounded P the P V product uses
-        sm.red[0][row] = psum / kappa + em * (zsum / esum);
-        sm.scl[0][row] = em / esum;
-      } else {
-        sm.red[1][row] = em * (zsum / esum);
-        sm.scl[1][row] = em / esum;
+        for (int cc = 0; cc < 2; ++cc)
+          *reinterpret_cast<uint4*>(prow + (((part * 2 + cc) ^ ((row >> 1) & 3)) << 4)) =
+              make_uint4(packed[4 * cc], packed[4 * cc + 1], packed[4 * cc + 2], packed[4 * cc + 3]);
       }
-      if (tc::named_barrier_any(1, 256, !good)) break;
-      const float den = sm.red[0][row] + sm.red[1][row];
-      const float cp = sm.scl[0][row], cm = sm.scl[1][row];
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sm.p_ready);
 
-      // epilogue: out = (c+ A+ + c- A-) / den for this thread's 64 columns.  After a failed
-      // wait here the warp skips it and meets the others at the next unit's barriers.
+      // X3: the partial sums of the rounded P (the denominator sums the same rounded P the
+      // P V product uses); the pair also agrees here whether to go on
+      mine[6 * kX] = psum;
+      if (tc::named_barrier_any(pair_bar, 64, !good)) break;
+      psum += theirs[6 * kX];
+      const float den = psum / kappa + em * (zsp / esp + zsm / esm);
+      const float cp = em / esp, cm = em / esm;
+
+      // epilogue: out = (c+ A+ + c- A-) / den for this warp's 64 columns.  After a failed
+      // wait here the warp skips it and meets its partner at the next unit's barriers.
       good = __all_sync(0xffffffffu, tc::mbar_wait(&sm.acc_full, k & 1, abort_flag, lim));
       if (!good) continue;
       tc::tc_fence_after();
       const float inv = den != 0.f ? 1.f / den : 0.f;
-      float ov[64];
-      {
+      uint32_t packed[32];  // this row's 64 output columns, bf16 pairs
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
         float a32[32], b32[32];
+        tc::tmem_ld32(tl + kColAp + part * 64 + h2 * 32, a32);
+        tc::tmem_ld32(tl + kColAm + part * 64 + h2 * 32, b32);
+        tc::tmem_wait_ld();
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          tc::tmem_ld32(tl + kColAp + half * 64 + h2 * 32, a32);
-          tc::tmem_ld32(tl + kColAm + half * 64 + h2 * 32, b32);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[h2 * 32 + i] = fmaf(cp, a32[i], cm * b32[i]) * inv;
-        }
+        for (int i = 0; i < 32; i += 2)
+          packed[h2 * 16 + i / 2] =
+              pack_bf16(fmaf(cp, a32[i], cm * b32[i]) * inv, fmaf(cp, a32[i + 1], cm * b32[i + 1]) * inv);
       }
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.acc_empty);
-      // This warp's 8 tokens x 4 heads x 64 columns are staged in its own 4 KiB buffer (staged
-      // row = lane = 4 * token + head; 16-byte chunk c at chunk c ^ (row % 8), the 128-byte
-      // swizzle) and written by one asynchronous bulk tensor store.  A warp whose tokens run
-      // past a short block writes its valid tokens with plain stores instead.  The buffer is
-      // reused one unit later, after the store has read it.
-      uint8_t* stg = sm.o[sw];
-      const int t0 = wq * 8;  // first token of this warp
-      if (t0 < x.n) {
-        if (lane == 0) tc::bulk_wait_read();
+      // 2 tokens x 4 heads x 64 columns at a time through 1 KiB of the (now idle) P buffer
+      // (16-byte chunk c of staged row r at chunk c ^ r), then each store instruction writes
+      // 4 rows x 128 contiguous bytes.  The pair stages inside the 2 KiB of P rows that only it
+      // writes, and it writes the next unit's P only after both warps have passed that unit's
+      // first pair barrier, so after these reads.
+      uint8_t* stg = sm.p + wq * 2048 + part * 1024;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if ((lane >> 3) == j) {
+          const int rr = lane & 7;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(stg + rr * 128 + ((c ^ rr) << 4)) =
+                make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+        }
         __syncwarp();
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 o4 = make_uint4(pack_bf16(ov[8 * c], ov[8 * c + 1]), pack_bf16(ov[8 * c + 2], ov[8 * c + 3]),
-                                      pack_bf16(ov[8 * c + 4], ov[8 * c + 5]), pack_bf16(ov[8 * c + 6], ov[8 * c + 7]));
-          *reinterpret_cast<uint4*>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) = o4;
+        for (int i = 0; i < 2; ++i) {
+          const int rr = 4 * i + (lane >> 3), c = lane & 7;
+          const uint4 o4 = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((c ^ rr) << 4));
+          const int grow = wq * 32 + 8 * j + rr;  // tile row
+          const int gt = grow >> 2, ghl = grow & 3;
+          if (gt < x.n)
+            *reinterpret_cast<uint4*>(p.O + ((size_t)(x.lo + gt) * p.Hq + kG * x.g + ghl) * kD + part * 64 + c * 8) = o4;
         }
-        tc::fence_proxy_async_smem();
         __syncwarp();
-        if (t0 + 8 <= x.n) {
-          if (lane == 0) {
-            tc::tma_store_3d(&p.tm_o, stg, half * 64, kG * x.g, x.lo + t0);
-            tc::bulk_commit();
-          }
-        } else {
-          const int hd = lane >> 3, c = lane & 7;
-          for (int tk = 0; t0 + tk < x.n; ++tk) {
-            const int rr = tk * kG + hd;
-            const uint4 o4 = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((c ^ (rr & 7)) << 4));
-            *reinterpret_cast<uint4*>(p.O + ((size_t)(x.lo + t0 + tk) * p.Hq + kG * x.g + hd) * kD + half * 64 + c * 8) = o4;
-          }
-        }
       }
     }
-    if (lane == 0) tc::bulk_wait_all();
   }
 
   tc::tc_fence_before();
@@ -583,8 +614,17 @@ cudaError_t launch_hybrid_tc(const HybridArgs& a, cudaStream_t st) {
   const int units = a.R * a.Hkv;
   int nsm = device_sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
-  int grid = nsm;
-  if (a.Hkv <= nsm) grid = (nsm / a.Hkv) * a.Hkv;  // keeps each CTA on one KV head
+  // Fewest CTAs that still finish in the same number of rounds (every CTA then takes the
+  // same number of units and a larger share of the memory bandwidth), kept a multiple of Hkv
+  // so that each CTA stays on one KV head.
+  const int rounds = (units + nsm - 1) / nsm;
+  int grid = (units + rounds - 1) / rounds;
+  if (a.Hkv <= nsm) {
+    grid = (grid + a.Hkv - 1) / a.Hkv * a.Hkv;
+    if (grid > nsm) grid = (nsm / a.Hkv) * a.Hkv;
+  } else {
+    grid = nsm;
+  }
   if (grid > units) grid = units;
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(hybrid_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
