@@ -29,14 +29,19 @@
 // Roles (320 threads):
 //   warp 0      TMA producer: Q/K and Z of unit k, then S of unit k as four stages of two
 //               32-row fp32 chunks (rows 32g.. of S+ and of S-; 128-byte swizzle with 32-byte
-//               atoms, the layout a tf32 MN-major operand needs) through a 3-stage ring, then V.
+//               atoms, the layout a tf32 MN-major operand needs) through a 4-stage ring that
+//               holds one whole unit, with V issued ahead of the last stage.
 //   warp 1      TMEM owner and MMA issuer (one thread): u = QW_g and s = QK^T (bf16), then
-//               A+/- += e S chunk by chunk (tf32, e from TMEM), then A+ += P V (bf16).
-//   warps 2-9   two threads per tile row (warps 2-5: the e+ half, warps 6-9: the e- half):
-//               block softmax, this half of e group by group (each group released to the
-//               MMA), the denominator parts, then the epilogue: each warp stages its 8 tokens
-//               x 4 heads x 64 columns in shared memory and writes them with one
-//               asynchronous bulk tensor store, whose completion it checks one unit later.
+//               A+ += e+ S+ and A- += e- S- group by group (tf32, e from TMEM), then
+//               A+ += P V (bf16).  The next unit's u and s are issued right behind, without
+//               waiting for these to complete (MMAs of one thread execute in issue order).
+//   warps 2-9   the two warps of each TMEM lane quarter share its 32 tile rows: warps 2-5
+//               take feature groups 0-1, block keys 0-15 and output columns 0-63, warps 6-9
+//               the rest.  Each computes e+ and e- of its groups from one read of u (each
+//               group released to the MMA as soon as it is in TMEM), its half of P, then its
+//               half of the epilogue, staged through the pair's own rows of the idle P buffer
+//               and written with coalesced 16-byte stores.  The pair exchanges per-row values
+//               through shared memory at three pair barriers per unit.
 //
 // Every wait is bounded; on expiry the CTA raises BHA_ERR_TIMEOUT in dev_err, drains its
 // own copies and MMAs, frees its TMEM and returns.
