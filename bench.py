@@ -82,11 +82,19 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def code_of(text):
+    """Source text with comments and blank space removed, so that a capture recorded for a
+    kernel stays valid across comment-only edits but not across code changes."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_hash(*names):
     h = hashlib.sha1()
     for n in names:
-        with open(os.path.join(ROOT, "linear_attention_diffusion_hedgehog_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "linear_attention_diffusion_hedgehog_b200", "csrc", n)) as f:
+            h.update(code_of(f.read()).encode())
     return h.hexdigest()[:12]
 
 
