@@ -465,10 +465,10 @@ def _line(metric, value, unit, args, world, ms_step, higher, config, **extra):
     return d
 
 
-def _roof(nbytes, ms, peaks, peak_src, kernel, flops=None):
+def _roof(nbytes, ms, peaks, peak_src, kernel, flops=None, traffic=None):
     achieved = nbytes / (ms / 1e3) / 1e9
     r = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-         "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+         "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
          "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": nbytes,
          "kernel": kernel}
     if flops is not None:
@@ -509,7 +509,9 @@ def bench_commit(args, world, rank, local):
                                R * B * world / (ms_step / 1e3), UNIT, args, world, ms_step, True, cfg,
                                dtype="bf16 in, fp32 state", kernel_variant=bha.kernel_variant(dims, 2),
                                roofline=_roof(commit_bytes(), ms_step, peaks, src, "commit",
-                                              flops=2 * R * HKV * B * (D * (F // 2) + F * D + F)),
+                                              flops=2 * R * HKV * B * (D * (F // 2) + F * D + F),
+                                              traffic=profiled_traffic("commit", source_hash("commit_tc.cu"))
+                                              if bha.kernel_variant(dims, 2) == 1 else None),
                                gpu_launches=args.steps)), flush=True)
 
 
