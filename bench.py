@@ -196,12 +196,20 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """The largest of the ranks' values (each rank's device time); the job's time is the
+    slowest rank's.  device is where the reduction tensor lives (cpu for gloo)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step, steps, max_ms, world):
+    """Units per second of the whole job: every rank processes units_per_rank_step units per
+    step (independent replicas, weak scaling) and the job takes the slowest rank's time."""
+    return units_per_rank_step * world * steps / (max_ms / 1e3)
 
 
 # ------------------------------------------------------------------ graph timing
@@ -383,8 +391,7 @@ def bench_decode(args, world, rank, local):
     clocks = sampler.stop(t0, t1) if rank == 0 else None
     ms = max_over_ranks(ms, world)
     step_ms = ms / args.steps
-    tokens = R * B * world * args.steps
-    value = tokens / (ms / 1e3)
+    value = whole_job_rate(R * B, args.steps, ms, world)
 
     # end to end through the public API: pinned host Q/K/V in, O back to pinned host
     e2e_steps = min(args.steps, 200)
@@ -418,7 +425,7 @@ def bench_decode(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    e2e_value = R * B * world * e2e_steps / (e2e_ms / 1e3)
+    e2e_value = whole_job_rate(R * B, e2e_steps, e2e_ms, world)
 
     if rank != 0:
         return
