@@ -75,7 +75,10 @@ typedef struct {
  *   x    [T][x_heads][d]  activation dtype;  head h uses W[floor(h * Hkv / x_heads)]
  *   W    [Hkv][d][F/2]    activation dtype
  *   phi  [T][x_heads][F]  out_dtype (BHA_F32 or BHA_BF16)
- * Uses dims->{num_kv_heads, head_dim, feature_dim, total_tokens, act_dtype}. */
+ * Uses dims->{num_kv_heads, head_dim, feature_dim, total_tokens, act_dtype}.
+ * bf16 x with d = 128, F = 256 and x_heads / num_kv_heads a power of two <= 128 (x_heads a
+ * multiple of num_kv_heads) takes the tensor-core kernel; its bounded waits have no error word
+ * here, so if one ever gave up the output of that call would be undefined (nothing traps). */
 int bha_featuremap(const bha_dims* dims, const void* x, int32_t x_heads, const void* W,
                    void* phi, int32_t out_dtype, void* stream);
 
@@ -145,8 +148,8 @@ int bha_full_prefix_attn_noalloc(const bha_dims* dims, const int32_t* cu_blk,
 const char* bha_status_string(int status);
 
 /* Which kernel variant a call with these dims takes: 0 = generic CUDA-core kernel,
- * 1 = tensor-core (tcgen05/TMA) kernel.  which: 0 featuremap, 1 hybrid, 2 commit,
- * 3 full prefix.  Negative on invalid dims. */
+ * 1 = tensor-core (tcgen05/TMA) kernel.  which: 0 featuremap (for x_heads = num_q_heads),
+ * 1 hybrid, 2 commit, 3 full prefix.  Negative on invalid dims. */
 int bha_kernel_variant(const bha_dims* dims, int32_t which);
 
 /* Library ABI version (major * 100 + minor). */

@@ -69,6 +69,9 @@ int bha_kernel_variant(const bha_dims* dims, int32_t which) {
   if (s != BHA_OK) return s;
   if (which < 0 || which > 3) return BHA_ERR_INVALID;
   const bool bf16 = dims->act_dtype == BHA_BF16;
+  if (which == 0)
+    return bha::featuremap_tc_supports(dims->total_tokens, dims->num_q_heads, dims->num_kv_heads,
+                                       dims->head_dim, dims->feature_dim, bf16) ? 1 : 0;
   if (which == 1) {
     bha::HybridArgs a{};
     a.R = dims->num_requests;
@@ -105,6 +108,11 @@ int bha_featuremap(const bha_dims* dims, const void* x, int32_t x_heads, const v
   if (dims->total_tokens == 0) return BHA_OK;
   if (!tensor_ok(x) || !tensor_ok(W) || !tensor_ok(phi)) return BHA_ERR_INVALID;
   if (x == phi || W == phi) return BHA_ERR_INVALID;
+  if (bha::featuremap_tc_supports(dims->total_tokens, x_heads, dims->num_kv_heads, dims->head_dim,
+                                  dims->feature_dim, dims->act_dtype == BHA_BF16))
+    return launch_status(bha::launch_featuremap_tc(x, dims->total_tokens, x_heads, dims->num_kv_heads,
+                                                   W, phi, out_dtype == BHA_BF16,
+                                                   static_cast<cudaStream_t>(stream)));
   return launch_status(bha::launch_featuremap_simt(
       x, dims->total_tokens, x_heads, dims->num_kv_heads, dims->head_dim, dims->feature_dim, W,
       phi, dims->act_dtype == BHA_BF16, out_dtype == BHA_BF16,

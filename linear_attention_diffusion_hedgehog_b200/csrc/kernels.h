@@ -89,6 +89,13 @@ struct TcFullParams {
   long long wait_limit;
 };
 
+// Parameters of the tensor-core feature-map kernel (featuremap_tc.cu).
+struct TcFeatParams {
+  CUtensorMap tm_x, tm_w, tm_o;
+  int T, H, Hw, G, out_bf16;
+  long long wait_limit;
+};
+
 // host helpers shared by the tensor-core launchers (tc_host.cu)
 enum TmaSwizzle { kTma128B, kTma128BAtom32, kTmaNone };
 bool make_tensor_map(CUtensorMap* m, bool f32, int rank, const void* base, const uint64_t* dims,
@@ -104,6 +111,9 @@ bool full_prefix_tc_supports(const FullPrefixArgs& a, bool act_bf16);
 int full_prefix_splits(int R, int Hkv, int64_t cap);
 size_t full_prefix_tc_workspace(const FullPrefixArgs& a);
 cudaError_t launch_full_prefix_tc(const FullPrefixArgs& a, void* workspace, cudaStream_t st);
+bool featuremap_tc_supports(int T, int x_heads, int Hw, int d, int F, bool act_bf16);
+cudaError_t launch_featuremap_tc(const void* x, int T, int x_heads, int Hw, const void* W, void* phi,
+                                 bool out_bf16, cudaStream_t st);
 
 // generic CUDA-core kernels (simt.cu)
 bool simt_supports(int d, int F, int Bmax);

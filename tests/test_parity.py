@@ -85,6 +85,61 @@ def test_featuremap_odd_dims_and_head_map():
     assert_close(host64(phi), ref.featuremap(c.Q, c.W), TOL_F32, "phi")
 
 
+def _check_phi(got, want, out_dt):
+    if out_dt == torch.float32:
+        assert_close(got, want, dict(rel_l2=1e-5, max_abs=1e-6), "phi")
+    else:  # bf16 output: one rounding of values in (0, 1)
+        assert_close(got, want, dict(rel_l2=5e-3, max_abs=4e-3), "phi")
+
+
+@pytest.mark.parametrize("H,Hkv,T", [(4, 4, 300), (16, 1, 77), (128, 1, 5), (64, 2, 33)])
+def test_featuremap_tensor_core_head_groupings(H, Hkv, T):
+    """G = H / Hkv heads per weight matrix from 1 to 128, so a warp's 32 output rows are 32
+    tokens of one head, several heads of several tokens, or a slice of one token's heads;
+    token counts that leave a ragged last tile (128 / G tokens per tile)."""
+    rng = np.random.default_rng(1000 * H + T)
+    x = inputs.bf16_round(rng.standard_normal((T, H, 128)).astype(np.float32))
+    W = inputs.bf16_round((rng.standard_normal((Hkv, 128, 128)) / np.sqrt(128)).astype(np.float32))
+    dims = bha.make_dims(0, H, Hkv, 128, 256, 1, T, 0, torch.bfloat16)
+    assert bha.kernel_variant(dims, 0) == 1
+    want = ref.featuremap(x, W)
+    for out_dt in (torch.float32, torch.bfloat16):
+        phi = bha.featuremap(dev(x, torch.bfloat16), dev(W, torch.bfloat16), out_dtype=out_dt)
+        torch.cuda.synchronize()
+        _check_phi(host64(phi), want, out_dt)
+
+
+def test_featuremap_group_size_not_a_power_of_two_takes_the_generic_kernel():
+    rng = np.random.default_rng(3)
+    x = inputs.bf16_round(rng.standard_normal((20, 12, 128)).astype(np.float32))
+    W = inputs.bf16_round((rng.standard_normal((4, 128, 128)) / np.sqrt(128)).astype(np.float32))
+    assert bha.kernel_variant(bha.make_dims(0, 12, 4, 128, 256, 1, 20, 0, torch.bfloat16), 0) == 0
+    phi = bha.featuremap(dev(x, torch.bfloat16), dev(W, torch.bfloat16))
+    torch.cuda.synchronize()
+    _check_phi(host64(phi), ref.featuremap(x, W), torch.float32)
+
+
+def test_featuremap_serving_size_sampled_rows():
+    """The bench's workload: x [4096, 16, 128] bf16, 4 weight matrices, fp32 phi; 64 sampled
+    (token, head) rows against the oracle, and every row's halves sum to 1."""
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(11)
+    x = torch.randn((4096, 16, 128), generator=gen, device="cuda").to(torch.bfloat16)
+    W = (torch.randn((4, 128, 128), generator=gen, device="cuda") / 128 ** 0.5).to(torch.bfloat16)
+    phi = bha.featuremap(x, W)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(12)
+    toks = rng.integers(0, 4096, 64)
+    heads = rng.integers(0, 16, 64)
+    xs = host64(x[toks, heads])
+    Wh = host64(W)
+    got = host64(phi[toks, heads])
+    want = np.stack([ref.phi(xs[i:i + 1], Wh[heads[i] // 4])[0] for i in range(64)])
+    _check_phi(got, want, torch.float32)
+    sums = phi.double().view(4096, 16, 2, 128).sum(-1)
+    assert torch.allclose(sums, torch.ones_like(sums), atol=1e-5)
+
+
 # ------------------------------------------------------------------- decode step, bf16
 
 def test_decode_step_one_layer_128_requests():
@@ -270,6 +325,8 @@ def test_tensor_core_path_is_taken_for_the_serving_shape():
     assert bha.kernel_variant(d, 2) == 1     # block commit on tensor cores
     assert bha.kernel_variant(d32, 2) == 0
     assert bha.kernel_variant(d, 3) == 1     # softmax teacher on tensor cores
+    assert bha.kernel_variant(d, 0) == 1     # feature map of the queries on tensor cores
+    assert bha.kernel_variant(d32, 0) == 0
 
 
 def test_linear_branch_dominant_states():
