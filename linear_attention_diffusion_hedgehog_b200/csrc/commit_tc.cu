@@ -16,7 +16,8 @@
 //                                 into one of two TMEM buffers
 //   S += dS, Z += dZ               fp32 read-modify-write by 8 warps: TMEM lane = d, so each
 //                                 warp instruction reads or writes one whole 128-byte line
-//                                 of a row of S; the other buffer's MMA overlaps it.
+//                                 of a row of S, 64 rows per thread in flight at a time;
+//                                 the other buffer's MMA overlaps it.
 // Computing dS transposed (lanes = d) is what makes the state update coalesced without
 // staging it through shared memory.
 //
@@ -351,16 +352,19 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
         tc::tc_fence_after();
         float* Sg = p.S + ((size_t)rq[j].slot * p.Hkv + g) * kF * kD;
         const uint32_t col0 = (b ? kColD1 : kColD0) + half * kFh;
+        // 64 state values per thread in flight at a time (64 KiB per CTA): the update is bound
+        // by the round trips of these loads, so each round moves as much as registers allow
 #pragma unroll 1
-        for (int fc = 0; fc < kFh / 32; ++fc) {
-          float dv[32], sv[32];
-          tc::tmem_ld32(tl + col0 + fc * 32, dv);
-          const int f0 = half * kFh + fc * 32;
+        for (int fc = 0; fc < kFh / 64; ++fc) {
+          float dv[64], sv[64];
+          const int f0 = half * kFh + fc * 64;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sv[i] = Sg[(size_t)(f0 + i) * kD + d];
+          for (int i = 0; i < 64; ++i) sv[i] = Sg[(size_t)(f0 + i) * kD + d];
+          tc::tmem_ld32(tl + col0 + fc * 64, *reinterpret_cast<float(*)[32]>(dv));
+          tc::tmem_ld32(tl + col0 + fc * 64 + 32, *reinterpret_cast<float(*)[32]>(dv + 32));
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) Sg[(size_t)(f0 + i) * kD + d] = sv[i] + dv[i];
+          for (int i = 0; i < 64; ++i) Sg[(size_t)(f0 + i) * kD + d] = sv[i] + dv[i];
         }
         float* Zg = p.Z + ((size_t)rq[j].slot * p.Hkv + g) * kF;
         Zg[tid] += sm.dz[j][tid];
