@@ -551,7 +551,9 @@ def bench_featuremap(args, world, rank, local):
         print(json.dumps(_line("feature-map rows/s", rows * world / (ms_step / 1e3), "rows/s", args,
                                world, ms_step, True, cfg, dtype="bf16 in, f32 out",
                                roofline=_roof(nbytes, ms_step, peaks, src, "featuremap",
-                                              flops=2 * rows * D * (F // 2)),
+                                              flops=2 * rows * D * (F // 2),
+                                              traffic=profiled_traffic("featuremap",
+                                                                       source_hash("featuremap_tc.cu"))),
                                gpu_launches=args.steps)), flush=True)
 
 
