@@ -31,17 +31,19 @@
 //               32-row fp32 chunks (rows 32g.. of S+ and of S-; 128-byte swizzle with 32-byte
 //               atoms, the layout a tf32 MN-major operand needs) through a 4-stage ring that
 //               holds one whole unit, with V issued ahead of the last stage.
-//   warp 1      TMEM owner and MMA issuer (one thread): u = QW_g and s = QK^T (bf16), then
-//               A+ += e+ S+ and A- += e- S- group by group (tf32, e from TMEM), then
-//               A+ += P V (bf16).  The next unit's u and s are issued right behind, without
-//               waiting for these to complete (MMAs of one thread execute in issue order).
-//   warps 2-9   the two warps of each TMEM lane quarter share its 32 tile rows: warps 2-5
-//               take feature groups 0-1, block keys 0-15 and output columns 0-63, warps 6-9
-//               the rest.  Each computes e+ and e- of its groups from one read of u (each
-//               group released to the MMA as soon as it is in TMEM), its half of P, then its
-//               half of the epilogue, staged through the pair's own rows of the idle P buffer
-//               and written with coalesced 16-byte stores.  The pair exchanges per-row values
-//               through shared memory at three pair barriers per unit.
+//   warp 1      TMEM owner and MMA issuer (one thread), per unit k: A+ += e+ S+ and
+//               A- += e- S- group by group (tf32, e from TMEM), then u = Q W_g and s = Q K^T of
+//               unit k+1 (bf16), then A+ += P V of unit k (bf16).  MMAs of one thread execute
+//               in issue order, so unit k+1's u and s overwrite e+ and the top of e- only after
+//               unit k's e S has read them, and unit k+1's feature map can start while unit k's
+//               P V is still waiting for its P.
+//   warps 2-5   feature map, one warp per TMEM lane quarter and one thread per tile row (its
+//               own TMEM lane): block-softmax max, e+ / e- group by group (each group released
+//               to the MMA as soon as the four warps have written it), P from the scores just
+//               before e- overwrites them, and the epilogue factors for the row.
+//   warps 6-9   epilogue, one warp per lane quarter: out = f+ A+ + f- A- once the unit's MMAs
+//               are done, each thread storing its row's 16-byte pieces straight from registers
+//               while the feature-map warps already work on the next unit.
 //
 // Every wait is bounded; on expiry the CTA raises BHA_ERR_TIMEOUT in dev_err, drains its
 // own copies and MMAs, frees its TMEM and returns.
@@ -92,13 +94,13 @@ struct __align__(1024) Smem {
                                    // 32-byte-atom swizzle
   uint8_t k[kKBytes];           // [d half][32 rows][128 B]
   uint8_t v[kKBytes];
-  uint8_t p[kPBytes];           // P: [128 rows][64 B], 64-byte swizzle; then output staging
+  uint8_t p[kPBytes];           // P: [128 rows][64 B], 64-byte swizzle
   float z[2][kF];
-  float xch[7][2][kM];          // per-row values the two warps of a lane quarter exchange
+  float fin[2][2][kM];          // per unit (double-buffered): epilogue factors c+/den, c-/den
   uint64_t qk_full, qk_empty, v_full, v_empty, v_ready, z_full[2], z_empty[2];
   uint64_t s_full[kStages], s_empty[kStages];
   uint64_t e_ready[kGroups], p_ready;
-  uint64_t w_full, u_full, acc_full, acc_empty, drain;
+  uint64_t w_full, u_full, acc_full, acc_empty, drain, fin_full[2], fin_empty[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -111,9 +113,9 @@ struct Unit {
 
 // Decodes unit u and validates it; every role calls this with the same arguments and so
 // skips the same units.
-// Order in which the S pairs are loaded and contracted: warps 2-5 produce groups 0 and 1
-// while warps 6-9 produce groups 2 and 3, so groups 0 and 2 become ready first.
-__device__ __forceinline__ int group_at(int i) { return (i & 1) * 2 + (i >> 1); }
+// Order in which the S pairs are loaded and contracted: the order the feature-map warps
+// produce the groups.
+__device__ __forceinline__ int group_at(int i) { return i; }
 
 __device__ __forceinline__ bool decode_unit(const TcHybridParams& p, int u, bool report, Unit* x) {
   x->g = u % p.Hkv;
@@ -150,21 +152,23 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
     tc::mbar_init(&sm.qk_empty, 1);
     tc::mbar_init(&sm.v_full, 1);
     tc::mbar_init(&sm.v_empty, 1);
-    tc::mbar_init(&sm.v_ready, 4);  // the four e+ warps clear V rows past a short block
+    tc::mbar_init(&sm.v_ready, 4);  // the four feature-map warps clear V rows past a short block
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&sm.z_full[i], 1);
-      tc::mbar_init(&sm.z_empty[i], 8);
+      tc::mbar_init(&sm.z_empty[i], 4);
+      tc::mbar_init(&sm.fin_full[i], 4);   // the four feature-map warps
+      tc::mbar_init(&sm.fin_empty[i], 4);  // the four epilogue warps
     }
-    for (int j = 0; j < kGroups; ++j) tc::mbar_init(&sm.e_ready[j], 4);  // the 4 warps owning group j
+    for (int j = 0; j < kGroups; ++j) tc::mbar_init(&sm.e_ready[j], 4);  // the 4 feature-map warps
     for (int i = 0; i < kStages; ++i) {
       tc::mbar_init(&sm.s_full[i], 1);
       tc::mbar_init(&sm.s_empty[i], 1);
     }
-    tc::mbar_init(&sm.p_ready, 8);
+    tc::mbar_init(&sm.p_ready, 4);
     tc::mbar_init(&sm.w_full, 1);
     tc::mbar_init(&sm.u_full, 1);
     tc::mbar_init(&sm.acc_full, 1);
-    tc::mbar_init(&sm.acc_empty, 8);
+    tc::mbar_init(&sm.acc_empty, 4);  // the four epilogue warps
     tc::mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     tc::fence_barrier_init();
@@ -257,26 +261,29 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Per unit k: A+/- += e S group by group, then the next unit's u and s, then A+ += P V.
+    // Issuing u(k+1) ahead of P V(k) lets the feature map of unit k+1 start as soon as the
+    // tensor pipe has finished e S(k), not after P V(k), which waits for unit k's P.  MMAs of
+    // one thread execute in issue order, so u(k+1) and s(k+1) overwrite e+ and the top of e-
+    // only after e S(k) has read them.
     if (lane == 0) {
       int g_res = -1, q = 0;
       uint32_t w_seen = 0;
       bool ok = true, issued = false;
       int ucur = blockIdx.x;
-      Unit x{};
-      for (int k = 0; ok && next_unit(p, units, &ucur, false, &x); ++k) {
-        if (x.g != g_res) {
-          if (!tc::mbar_wait(&sm.w_full, w_seen & 1, abort_flag, lim)) { ok = false; break; }
+      Unit x{}, xn{};
+      const uint32_t wa = tc::smem_u32(sm.w);
+      const uint32_t qa = tc::smem_u32(sm.q);
+      const uint32_t ka = tc::smem_u32(sm.k);
+      // u = Q W_g and s = Q K^T of unit j
+      auto issue_uqk = [&](const Unit& y, int j) -> bool {
+        if (y.g != g_res) {
+          if (!tc::mbar_wait(&sm.w_full, w_seen & 1, abort_flag, lim)) return false;
           ++w_seen;
-          g_res = x.g;
+          g_res = y.g;
         }
-        // u and the scores overwrite e+ and the top of e-, which the previous unit's MMAs read
-        // as their A operand: MMAs issued by one thread execute in issue order, so these are
-        // issued right behind them without waiting for them to complete
-        if (!tc::mbar_wait(&sm.qk_full, k & 1, abort_flag, lim)) { ok = false; break; }
+        if (!tc::mbar_wait(&sm.qk_full, j & 1, abort_flag, lim)) return false;
         tc::tc_fence_after();
-        const uint32_t qa = tc::smem_u32(sm.q);
-        const uint32_t wa = tc::smem_u32(sm.w);
-        const uint32_t ka = tc::smem_u32(sm.k);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t a = tc::smem_desc(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
@@ -292,10 +299,14 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
         tc::mma_commit(&sm.u_full);
         tc::mma_commit(&sm.qk_empty);
         issued = true;
+        return true;
+      };
+      bool have = next_unit(p, units, &ucur, false, &x);
+      if (have) ok = issue_uqk(x, 0);
+      for (int k = 0; ok && have; ++k) {
         // the accumulators are free once the previous epilogue has read them
         if (k >= 1 && !tc::mbar_wait(&sm.acc_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
         // A+ += e+ S+ and A- += e- S-, group by group as the feature-map warps release them
-        // (one wait per group for both halves keeps this thread's per-MMA overhead low)
         for (int i = 0; i < kGroups; ++i, ++q) {
           const int grp = group_at(i);
           if (!tc::mbar_wait(&sm.e_ready[grp], k & 1, abort_flag, lim)) { ok = false; break; }
@@ -317,6 +328,9 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
           tc::mma_commit(&sm.s_empty[st]);
         }
         if (!ok) break;
+        // the next unit's u and s
+        const bool have_next = next_unit(p, units, &ucur, false, &xn);
+        if (have_next && !issue_uqk(xn, k + 1)) { ok = false; break; }
         // A+ += P V
         if (!tc::mbar_wait(&sm.p_ready, k & 1, abort_flag, lim)) { ok = false; break; }
         if (!tc::mbar_wait(&sm.v_ready, k & 1, abort_flag, lim)) { ok = false; break; }
@@ -331,6 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
         }
         tc::mma_commit(&sm.v_empty);
         tc::mma_commit(&sm.acc_full);
+        x = xn;
+        have = have_next;
       }
       if (issued) {
         volatile int never = 0;
@@ -338,90 +354,68 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
         tc::mbar_wait(&sm.drain, 0, &never, lim);
       }
     }
-  } else {
-    // ------------------------------------------------------------ feature map / epilogue
-    // The two warps of a TMEM lane quarter share its 32 tile rows: warp part 0 (warps 2-5)
-    // takes feature groups 0 and 1 of u, part 1 (warps 6-9) groups 2 and 3; each computes both
-    // e+ and e- of its groups from one read of u, half of the block keys of P, and half of
-    // the output columns.  They exchange per-row values through shared memory at three pair
-    // barriers per unit (X1: max/min of u, X2: partial sums, X3: partial P sum).
-    const int sw = warp - 2;           // 0..7
-    const int part = sw >> 2;          // 0: groups 0-1, keys 0-15, columns 0-63; 1: the rest
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ feature map
+    // One warp per TMEM lane quarter, one thread per tile row (its own TMEM lane).  A failed
+    // bounded wait ends the loop for the whole warp (the vote keeps its lanes together).
     const int wq = warp & 3;           // TMEM lane quarter this warp may access
     const int row = wq * 32 + lane;    // tile row = 4 t + head-in-group
     const int hl = row & 3;
     const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
-    const uint32_t pair_bar = 2 + wq;
     const float scale_log2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
     const float log2e = 1.4426950408889634f;
-    const int g0 = part * 2;           // this warp's first feature group
-    float* mine = &sm.xch[0][part][row];
-    const float* theirs = &sm.xch[0][part ^ 1][row];
-    constexpr int kX = 2 * kM;         // stride between exchange slots
     int ucur = blockIdx.x;
     Unit x{};
-    // A failed wait does not leave the loop at once: the two warps of a pair meet at named
-    // barriers, so both finish the unit's barriers and leave together, decided by the
-    // reducing barrier at its end.  Work done after a failed wait is discarded.
-    bool good = true;
     for (int k = 0; next_unit(p, units, &ucur, false, &x); ++k) {
-      good = tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim) && good;
-      good = tc::mbar_wait(&sm.z_full[k & 1], (k >> 1) & 1, abort_flag, lim) && good;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim))) break;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.z_full[k & 1], (k >> 1) & 1, abort_flag, lim))) break;
       tc::tc_fence_after();
 
-      float sv[32], u0[32], u1[32];
-      tc::tmem_ld32(tl + kColS, sv);
-      tc::tmem_ld32(tl + kColU + g0 * 32, u0);
-      tc::tmem_ld32(tl + kColU + g0 * 32 + 32, u1);
-      tc::tmem_wait_ld();
-
       // block softmax over the x.n keys of this request (bidirectional, no mask):
-      // a_j = w 2^{s_j log2e / sqrt d - m}; this warp keeps its 16 keys in fp32 until P's
-      // scale is known
-      float av[16];
+      // a_j = w 2^{s_j log2e / sqrt d - m}; here only the row max m, P itself is formed once
+      // P's scale is known (below, from the scores still in TMEM)
       float m2;
       {
+        float sv[32];
+        tc::tmem_ld32(tl + kColS, sv);
+        tc::tmem_wait_ld();
         float mraw = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           if (j < x.n) mraw = fmaxf(mraw, sv[j]);
         // m in log2 units, kept in [-6 log2 e, 90] so that 2^{-m} is finite and not tiny
         m2 = fminf(fmaxf(mraw * scale_log2, -6.f * log2e), 90.f);
-        const float wgt = p.alpha ? 1.f / (1.f + expf(-p.alpha[kG * x.g + hl])) : 1.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int jj = part * 16 + j;
-          const float s_j = part ? sv[16 + j] : sv[j];
-          av[j] = jj < x.n ? wgt * tc::ex2(fmaf(s_j, scale_log2, -m2)) : 0.f;
-        }
       }
+      const float wgt = p.alpha ? 1.f / (1.f + expf(-p.alpha[kG * x.g + hl])) : 1.f;
       const float em = tc::ex2(-m2);
 
-      // X1: max and min of u over the row's 128 features
+      // max and min of u over the row's 128 features
       float mx = -INFINITY, mn = INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < kGroups; c += 2) {
+        float u0[32], u1[32];
+        tc::tmem_ld32(tl + kColU + c * 32, u0);
+        tc::tmem_ld32(tl + kColU + c * 32 + 32, u1);
+        tc::tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        mx = fmaxf(mx, fmaxf(u0[i], u1[i]));
-        mn = fminf(mn, fminf(u0[i], u1[i]));
+        for (int i = 0; i < 32; ++i) {
+          mx = fmaxf(mx, fmaxf(u0[i], u1[i]));
+          mn = fminf(mn, fminf(u0[i], u1[i]));
+        }
       }
-      mine[0 * kX] = mx;
-      mine[1 * kX] = mn;
-      // (both warps have also read the scores, which e- group 3 overwrites, by this barrier)
-      tc::tc_fence_before();
-      tc::named_barrier_sync(pair_bar, 64);
-      tc::tc_fence_after();
-      mx = fmaxf(mx, theirs[0 * kX]);
-      mn = fminf(mn, theirs[1 * kX]);
 
       // e+_f = 2^{(u_f - max u) log2e} over u in place, e-_f = 2^{(min u - u_f) log2e}, group by
-      // group, each released to the MMA as soon as the four warps owning it have written it
+      // group, each released to the MMA as soon as the four warps have written it (e- group 3
+      // overwrites the scores, which this thread has read)
       const float bpl = mx * log2e, bml = mn * log2e;
       const float* zk = sm.z[k & 1];
-      float esp = 0.f, esm = 0.f, zsp = 0.f, zsm = 0.f;
-#pragma unroll
-      for (int gi = 0; gi < 2; ++gi) {
-        float(&uu)[32] = gi ? u1 : u0;
-        const int c = g0 + gi;
+      float esp = 0.f, esm = 0.f, zsp = 0.f, zsm = 0.f, kappa = 1.f, psum = 0.f;
+      bool vgood = true;
+#pragma unroll 1
+      for (int c = 0; c < kGroups; ++c) {
+        float uu[32];
+        tc::tmem_ld32(tl + kColU + c * 32, uu);
+        tc::tmem_wait_ld();
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           float ep[16];
@@ -439,6 +433,31 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
           }
           tc::tmem_st16(tl + kColU + c * 32 + 16 * h, ep);
         }
+        if (c == kGroups - 1) {
+          // sum e+ is complete, so P (bf16, scaled by kappa = sum e+ / e^{-m}) is formed now,
+          // from the scores that e- group 3 is about to overwrite.  P's buffer is free once
+          // V has landed (V is reloaded only after the previous P V has completed).
+          vgood = __all_sync(0xffffffffu, tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim));
+          kappa = esp / em;
+          float sv[32];
+          tc::tmem_ld32(tl + kColS, sv);
+          tc::tmem_wait_ld();
+          uint32_t packed[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float a0 = j < x.n ? wgt * tc::ex2(fmaf(sv[j], scale_log2, -m2)) : 0.f;
+            const float a1 = j + 1 < x.n ? wgt * tc::ex2(fmaf(sv[j + 1], scale_log2, -m2)) : 0.f;
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(a0 * kappa, a1 * kappa);
+            psum += __low2float(b2) + __high2float(b2);
+            packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          // 64-byte rows, 16-byte chunk c stored at chunk c ^ ((row / 2) % 4) (64-byte swizzle)
+          uint8_t* prow = sm.p + row * 64;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            *reinterpret_cast<uint4*>(prow + ((q4 ^ ((row >> 1) & 3)) << 4)) =
+                make_uint4(packed[4 * q4], packed[4 * q4 + 1], packed[4 * q4 + 2], packed[4 * q4 + 3]);
+        }
         tc::tmem_st32(tl + kColEm + c * 32, uu);
         tc::tmem_wait_st();
         tc::tc_fence_before();
@@ -447,111 +466,81 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
       }
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.z_empty[k & 1]);
+      if (!vgood) break;
 
-      // X2: the partial sums
-      mine[2 * kX] = esp;
-      mine[3 * kX] = esm;
-      mine[4 * kX] = zsp;
-      mine[5 * kX] = zsm;
-      tc::named_barrier_sync(pair_bar, 64);
-      esp += theirs[2 * kX];
-      esm += theirs[3 * kX];
-      zsp += theirs[4 * kX];
-      zsm += theirs[5 * kX];
-
-      if (part == 0) {
-        // V of this unit: rows past a short block belong to another request; clear them
-        good = tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim) && good;
-        if (x.n < kBlk) {
-          const int per_half = (kBlk - x.n) * 8;
-          for (int i = sw * 32 + lane; i < 2 * per_half; i += 128) {
-            const int hh = i / per_half, rem = i % per_half;
-            *reinterpret_cast<uint4*>(sm.v + hh * (kKBytes / 2) + (x.n + rem / 8) * 128 + (rem % 8) * 16) =
-                make_uint4(0, 0, 0, 0);
-          }
+      // V of this unit: rows past a short block belong to another request; clear them
+      if (x.n < kBlk) {
+        const int per_half = (kBlk - x.n) * 8;
+        for (int i = wq * 32 + lane; i < 2 * per_half; i += 128) {
+          const int hh = i / per_half, rem = i % per_half;
+          *reinterpret_cast<uint4*>(sm.v + hh * (kKBytes / 2) + (x.n + rem / 8) * 128 + (rem % 8) * 16) =
+              make_uint4(0, 0, 0, 0);
         }
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&sm.v_ready);
-      }
-
-      // P (bf16, scaled by kappa = sum e+ / e^{-m}): this warp's 16 keys, two 16-byte chunks of
-      // the row's 64 bytes (chunk c stored at chunk c ^ ((row / 2) % 4), the 64-byte swizzle)
-      const float kappa = esp / em;
-      float psum = 0.f;
-      {
-        uint32_t packed[8];
-#pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(av[j] * kappa, av[j + 1] * kappa);
-          psum += __low2float(b2) + __high2float(b2);
-          packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
-        }
-        uint8_t* prow = sm.p + row * 64;
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc)
-          *reinterpret_cast<uint4*>(prow + (((part * 2 + cc) ^ ((row >> 1) & 3)) << 4)) =
-              make_uint4(packed[4 * cc], packed[4 * cc + 1], packed[4 * cc + 2], packed[4 * cc + 3]);
       }
       tc::fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sm.p_ready);
-
-      // X3: the partial sums of the rounded P (the denominator sums the same rounded P the
-      // P V product uses); the pair also agrees here whether to go on
-      mine[6 * kX] = psum;
-      if (tc::named_barrier_any(pair_bar, 64, !good)) break;
-      psum += theirs[6 * kX];
-      const float den = psum / kappa + em * (zsp / esp + zsm / esm);
-      const float cp = em / esp, cm = em / esm;
-
-      // epilogue: out = (c+ A+ + c- A-) / den for this warp's 64 columns.  After a failed
-      // wait here the warp skips it and meets its partner at the next unit's barriers.
-      good = __all_sync(0xffffffffu, tc::mbar_wait(&sm.acc_full, k & 1, abort_flag, lim));
-      if (!good) continue;
-      tc::tc_fence_after();
-      const float inv = den != 0.f ? 1.f / den : 0.f;
-      uint32_t packed[32];  // this row's 64 output columns, bf16 pairs
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        float a32[32], b32[32];
-        tc::tmem_ld32(tl + kColAp + part * 64 + h2 * 32, a32);
-        tc::tmem_ld32(tl + kColAm + part * 64 + h2 * 32, b32);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; i += 2)
-          packed[h2 * 16 + i / 2] =
-              pack_bf16(fmaf(cp, a32[i], cm * b32[i]) * inv, fmaf(cp, a32[i + 1], cm * b32[i + 1]) * inv);
+      if (lane == 0) {
+        tc::mbar_arrive(&sm.v_ready);
+        tc::mbar_arrive(&sm.p_ready);
       }
-      tc::tc_fence_before();
+
+      // epilogue factors: out = (c+ A+ + c- A-) / den, c+/- = e^{-m} / sum e+/-,
+      // den = w sum_j P_j + e^{-m} (e+.Z+ / sum e+ + e-.Z- / sum e-) with the same rounded P
+      // that the P V product uses; handed to the epilogue warps through a double buffer
+      const int fb = k & 1;
+      if (k >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(&sm.fin_empty[fb], ((k - 2) >> 1) & 1, abort_flag, lim)))
+        break;
+      const float den = psum / kappa + em * (zsp / esp + zsm / esm);
+      const float inv = den != 0.f ? 1.f / den : 0.f;
+      sm.fin[fb][0][row] = em / esp * inv;
+      sm.fin[fb][1][row] = em / esm * inv;
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sm.acc_empty);
-      // 2 tokens x 4 heads x 64 columns at a time through 1 KiB of the (now idle) P buffer
-      // (16-byte chunk c of staged row r at chunk c ^ r), then each store instruction writes
-      // 4 rows x 128 contiguous bytes.  The pair stages inside the 2 KiB of P rows that only it
-      // writes, and it writes the next unit's P only after both warps have passed that unit's
-      // first pair barrier, so after these reads.
-      uint8_t* stg = sm.p + wq * 2048 + part * 1024;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if ((lane >> 3) == j) {
-          const int rr = lane & 7;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(stg + rr * 128 + ((c ^ rr) << 4)) =
-                make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+      if (lane == 0) tc::mbar_arrive(&sm.fin_full[fb]);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // One warp per TMEM lane quarter: out = f+ A+ + f- A- for its 32 rows, written straight
+    // from registers (each thread its row's 64-byte chunks) while the feature-map warps
+    // already work on the next unit.
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const int tok = row >> 2, hl = row & 3;
+    const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
+    int ucur = blockIdx.x;
+    Unit x{};
+    for (int k = 0; next_unit(p, units, &ucur, false, &x); ++k) {
+      const int fb = k & 1;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.acc_full, k & 1, abort_flag, lim))) break;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.fin_full[fb], (k >> 1) & 1, abort_flag, lim))) break;
+      tc::tc_fence_after();
+      const float fp = sm.fin[fb][0][row], fm = sm.fin[fb][1][row];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&sm.fin_empty[fb]);
+      __nv_bfloat16* orow = p.O + ((size_t)(x.lo + tok) * p.Hq + kG * x.g + hl) * kD;
+      const bool live = tok < x.n;
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        float a32[32], b32[32];
+        tc::tmem_ld32(tl + kColAp + c * 32, a32);
+        tc::tmem_ld32(tl + kColAm + c * 32, b32);
+        tc::tmem_wait_ld();
+        if (c == kD / 32 - 1) {
+          // every read of the accumulators is done: the next unit's MMAs may overwrite them
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&sm.acc_empty);
         }
-        __syncwarp();
+        if (live) {
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int rr = 4 * i + (lane >> 3), c = lane & 7;
-          const uint4 o4 = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((c ^ rr) << 4));
-          const int grow = wq * 32 + 8 * j + rr;  // tile row
-          const int gt = grow >> 2, ghl = grow & 3;
-          if (gt < x.n)
-            *reinterpret_cast<uint4*>(p.O + ((size_t)(x.lo + gt) * p.Hq + kG * x.g + ghl) * kD + part * 64 + c * 8) = o4;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            float o[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) o[j] = fmaf(fp, a32[8 * q4 + j], fm * b32[8 * q4 + j]);
+            *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) =
+                make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
+                           pack_bf16(o[6], o[7]));
+          }
         }
-        __syncwarp();
       }
     }
   }
