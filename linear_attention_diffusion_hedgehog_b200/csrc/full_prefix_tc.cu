@@ -387,16 +387,32 @@ bool full_prefix_tc_supports(const FullPrefixArgs& a, bool act_bf16) {
 
 // Number of KV splits per (request, KV head): enough units to cover the SMs several times,
 // each split at least 4 tiles long.  Depends only on the call's dims and cache capacity.
+// Number of key-range splits per (request, KV head).  Cost model in units of one 128-key
+// K/V tile (64 KiB): a unit of work costs its tiles plus its 32 KiB Q tile and 32 KiB output
+// (1 tile), and with splits also its fp32 partial output written and read back by the
+// combine step (about 2 more tiles); the grid runs ceil(units / SMs) rounds.  The split count
+// with the least (rounds x cost per unit) wins, keeping at least 4 tiles per split.  The SM
+// count is fixed at 148 so that the workspace size does not depend on the device.
 int full_prefix_splits(int R, int Hkv, int64_t cap) {
   const long long pairs = (long long)R * Hkv;
   const long long tiles = (cap + kKT - 1) / kKT;
   if (pairs <= 0 || tiles <= 0) return 1;
-  long long want = (148 * 8 + pairs - 1) / pairs;
+  const long long nsm = 148;
   long long most = (tiles + 3) / 4;
-  long long s = want < most ? want : most;
-  if (s < 1) s = 1;
-  if (s > 64) s = 64;
-  return (int)s;
+  if (most > 64) most = 64;
+  if (most < 1) most = 1;
+  long long best = 1;
+  double best_cost = 0.0;
+  for (long long s = 1; s <= most; ++s) {
+    const long long rounds = (pairs * s + nsm - 1) / nsm;
+    const double per_unit = (double)((tiles + s - 1) / s) + (s == 1 ? 1.0 : 3.1);
+    const double cost = (double)rounds * per_unit;
+    if (s == 1 || cost < best_cost) {
+      best = s;
+      best_cost = cost;
+    }
+  }
+  return (int)best;
 }
 
 size_t full_prefix_tc_workspace(const FullPrefixArgs& a) {
@@ -447,7 +463,10 @@ cudaError_t launch_full_prefix_tc(const FullPrefixArgs& a, void* workspace, cuda
   const int units = a.R * a.Hkv * p.nsplit;
   int nsm = device_sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
-  const int grid = units < nsm ? units : nsm;
+  // fewest CTAs that finish in the same number of rounds
+  const int rounds = (units + nsm - 1) / nsm;
+  int grid = (units + rounds - 1) / rounds;
+  if (grid > nsm) grid = nsm;
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(full_prefix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
