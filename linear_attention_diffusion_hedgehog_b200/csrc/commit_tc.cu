@@ -254,6 +254,11 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
     const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
     const float log2e = 1.4426950408889634f;
     int k = 0, rc = 0;
+    // A failed wait does not leave the loop at once: these 256 threads meet at a named barrier
+    // each unit, so all of them reach it and leave together, decided by the reducing barrier.
+    // Work done after a failed wait goes no further than shared memory (S and Z are not
+    // written).
+    bool good = true;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       const int g = u % p.Hkv, j0 = (u / p.Hkv) * kReq;
       Req rq[kReq];
@@ -262,8 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
 #pragma unroll
       for (int j = 0; j < kReq; ++j) nreq += rq[j].n > 0;
       if (nreq == 0) continue;
-      if (!tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim)) break;
-      if (!tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim)) break;
+      good = tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim) && good;
+      good = tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim) && good;
       tc::tc_fence_after();
       // ---- this thread's half of phi for key row `row`, rounded to bf16
       const int jr = row >> 5, t = row & 31;
@@ -319,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
         }
       }
       tc::tc_fence_before();
-      tc::named_barrier_sync(1, 256);
+      if (tc::named_barrier_any(1, 256, !good)) break;
       tc::tc_fence_after();
       // ---- dZ[j][f] = sum over the block's tokens of the bf16 phi (thread tid owns f = tid)
       {
@@ -348,7 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
       for (int j = 0; j < kReq; ++j) {
         if (rq[j].n == 0) continue;
         const int b = rc & 1;
-        if (!tc::mbar_wait(&sm.d_full[b], (rc >> 1) & 1, abort_flag, lim)) { k = -1; break; }
+        // (a failed wait skips this unit's remaining updates; the next barrier ends the loop)
+        good = __all_sync(0xffffffffu, tc::mbar_wait(&sm.d_full[b], (rc >> 1) & 1, abort_flag, lim));
+        if (!good) break;
         tc::tc_fence_after();
         float* Sg = p.S + ((size_t)rq[j].slot * p.Hkv + g) * kF * kD;
         const uint32_t col0 = (b ? kColD1 : kColD0) + half * kFh;
@@ -373,7 +380,6 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
         if (lane == 0) tc::mbar_arrive(&sm.d_empty[b]);
         ++rc;
       }
-      if (k < 0) break;
       ++k;
     }
   }
