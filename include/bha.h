@@ -144,6 +144,14 @@ int bha_full_prefix_attn_noalloc(const bha_dims* dims, const int32_t* cu_blk,
                                  const void* Vc, int64_t kv_capacity, void* O, int32_t* dev_err,
                                  void* stream);
 
+/* Self-test of the watchdog that bounds every wait inside the tensor-core kernels: launches
+ * one CTA whose thread waits, through that same bounded wait, on an mbarrier nothing ever
+ * arrives at.  After about limit_cycles SM cycles (1 .. 4e9) the wait gives up and the kernel
+ * writes BHA_ERR_TIMEOUT to *dev_err (a DEVICE int32 the caller zeroes first), as a stalled
+ * pipeline would; the context stays usable.  Returns BHA_ERR_INVALID for a NULL dev_err or a
+ * limit out of range, else the launch status. */
+int bha_selftest_bounded_wait(int64_t limit_cycles, int32_t* dev_err, void* stream);
+
 /* Static description of a status code. */
 const char* bha_status_string(int status);
 

@@ -58,6 +58,7 @@ _SIGS = {
     "bha_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bha_kernel_variant": (ctypes.c_int, [ctypes.POINTER(Dims), _I32]),
     "bha_version": (ctypes.c_int, []),
+    "bha_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_int64, _P, _P]),
 }
 
 _lib = None
@@ -85,6 +86,15 @@ def header_functions() -> list[str]:
     src = open(HEADER_PATH).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(bha_\w+)\s*\(", src)))
+
+
+def selftest_bounded_wait(limit_cycles, dev_err, stream=None):
+    """Runs the library's bounded wait on an mbarrier that never completes; dev_err (a device
+    int32 tensor, zeroed by the caller) receives BHA_ERR_TIMEOUT once the wait gives up."""
+    _cuda(dev_err, "dev_err", dtype=torch.int32)
+    st = lib().bha_selftest_bounded_wait(int(limit_cycles), _ptr(dev_err),
+                                         _stream(dev_err.device, stream))
+    _check(st, "bha_selftest_bounded_wait")
 
 
 def status_string(status: int) -> str:

@@ -128,3 +128,11 @@ def test_kernel_variant_query():
     assert bha.kernel_variant(dims(), 1) in (0, 1)
     assert bha.kernel_variant(dims(F=3), 1) == bha.BHA_ERR_INVALID
     assert bha.kernel_variant(dims(), 9) == bha.BHA_ERR_INVALID
+
+
+def test_selftest_bounded_wait_rejects_bad_arguments_before_launching():
+    L = bha.lib()
+    assert L.bha_selftest_bounded_wait(1000, None, None) == -1      # no dev_err
+    dummy = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    assert L.bha_selftest_bounded_wait(0, dummy, None) == -1        # limit below range
+    assert L.bha_selftest_bounded_wait(5_000_000_000, dummy, None) == -1  # above range

@@ -410,3 +410,21 @@ def test_full_prefix_teacher_serving_size_sampled():
         sl = slice(32 * r, 32 * r + 32)
         want = ref.full_prefix_attn([0, 32], [L], Qh[sl], Kh[r:r + 1], Vh[r:r + 1])
         assert_close(O[sl], want, TOL_BF16, f"O[{r}]")
+
+
+# ------------------------------------------------------------------- watchdog
+
+def test_bounded_wait_gives_up_and_reports_timeout():
+    """The bounded wait every tensor-core kernel uses, on an mbarrier nothing arrives at:
+    after its limit it reports BHA_ERR_TIMEOUT through dev_err and the context stays usable
+    (a feature map right after runs and matches the oracle)."""
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bha.selftest_bounded_wait(2_000_000, err)  # about a millisecond of SM cycles
+    torch.cuda.synchronize()
+    assert int(err.item()) == -4, bha.status_string(int(err.item()))
+    rng = np.random.default_rng(8)
+    x = inputs.bf16_round(rng.standard_normal((40, 8, 128)).astype(np.float32))
+    W = inputs.bf16_round((rng.standard_normal((2, 128, 128)) / np.sqrt(128)).astype(np.float32))
+    phi = bha.featuremap(dev(x, torch.bfloat16), dev(W, torch.bfloat16))
+    torch.cuda.synchronize()
+    _check_phi(host64(phi), ref.featuremap(x, W), torch.float32)
