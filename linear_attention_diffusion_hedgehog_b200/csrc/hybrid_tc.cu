@@ -179,7 +179,6 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
     tc::prefetch_tensormap(&p.tm_v);
     tc::prefetch_tensormap(&p.tm_w);
     tc::prefetch_tensormap(&p.tm_s);
-    tc::prefetch_tensormap(&p.tm_o);
   }
   if (warp == 1) {
     tc::tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -568,8 +567,6 @@ cudaError_t launch_hybrid_tc(const HybridArgs& a, cudaStream_t st) {
     const uint64_t strides[2] = {kD * 2, (uint64_t)a.Hq * kD * 2};
     const uint32_t box[3] = {64, kG, kBlk};
     if (!make_tensor_map(&p.tm_q, false, 3, a.Q, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
-    const uint32_t obox[3] = {64, kG, 8};
-    if (!make_tensor_map(&p.tm_o, false, 3, a.O, dims, strides, obox, kTma128B)) return cudaErrorInvalidValue;
   }
   {
     const uint64_t dims[3] = {kD, (uint64_t)a.Hkv, T};

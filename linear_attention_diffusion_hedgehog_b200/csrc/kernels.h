@@ -52,7 +52,7 @@ struct FullPrefixArgs {
 // Parameters of the tensor-core decode-step kernel (hybrid_tc.cu); the tensor maps describe
 // Q, K, V, W and S for the Tensor Memory Accelerator.
 struct TcHybridParams {
-  CUtensorMap tm_q, tm_k, tm_v, tm_w, tm_s, tm_o;
+  CUtensorMap tm_q, tm_k, tm_v, tm_w, tm_s;
   const int32_t* cu_blk;
   const int32_t* state_slot;
   const float* Z;
