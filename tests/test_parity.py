@@ -159,6 +159,41 @@ def test_decode_step_one_layer_128_requests():
     assert_close(host64(O)[rows], want[rows], TOL_BF16, "O")
 
 
+def test_decode_step_and_commit_1024_requests_many_units_per_cta():
+    """1024 requests (4096 (request, KV head) units: about 28 per CTA for the decode step, and
+    1024 four-request units for the commits that build the 64-token prefixes), so each CTA
+    walks many units with its buffers and W_g reused; 8 sampled requests checked in full."""
+    c = inputs.decode_case(R=1024, Hq=16, Hkv=4, d=128, F=256, block_lens=32, prefix_lens=64,
+                           seed=31, dtype="bf16")
+    S, Z = build_states_on_gpu(c, block=32)
+    O = run_hybrid(c, S, Z)
+    reqs = np.random.default_rng(5).choice(1024, 8, replace=False)
+    So, Zo = oracle_states(c, reqs)
+    Oh = host64(O)
+    for r in reqs:
+        assert_close(host64(S[r]), So[r], TOL_BF16, f"S[{r}]")
+        assert_close(host64(Z[r]), Zo[r], TOL_BF16, f"Z[{r}]")
+        lo, hi = c.cu_blk[r], c.cu_blk[r + 1]
+        want = ref.hybrid_attn([0, hi - lo], c.Q[lo:hi], c.K[lo:hi], c.V[lo:hi], So[r:r + 1],
+                               Zo[r:r + 1], c.W)
+        assert_close(Oh[lo:hi], want, TOL_BF16, f"O[{r}]")
+
+
+def test_decode_step_three_kv_heads_grid_stays_on_one_weight():
+    """Hkv = 3 (12 query heads), 50 requests: 150 units on a grid sized to a multiple of 3, so
+    every CTA keeps one W_g; ragged blocks and prefixes; every row checked."""
+    lens = np.random.default_rng(2).integers(1, 33, 50)
+    c = inputs.decode_case(R=50, Hq=12, Hkv=3, d=128, F=256, block_lens=lens, prefix_lens=64,
+                           seed=32, dtype="bf16")
+    d = bha.make_dims(50, 12, 3, 128, 256, 32, int(c.cu_blk[-1]), 50, torch.bfloat16)
+    assert bha.kernel_variant(d, 1) == 1
+    S, Z = build_states_on_gpu(c, block=32)
+    O = run_hybrid(c, S, Z)
+    So, Zo = oracle_states(c)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, So, Zo, c.W)
+    assert_close(host64(O), want, TOL_BF16, "O")
+
+
 def test_decode_step_ragged_slots_gate_isolated_states():
     """Ragged blocks (0, 1, 31, 32 tokens), a permuted slot map, the sigmoid gate, and
     directly drawn states, so the cross-block read is checked on its own."""
