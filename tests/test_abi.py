@@ -3,6 +3,7 @@ declares, and rejects bad arguments on the host before launching anything.  No c
 reaches a kernel: each one either fails validation or has no work (R = 0 / T = 0), so the
 suite runs without a GPU."""
 import ctypes
+import os
 
 import pytest
 
@@ -136,3 +137,19 @@ def test_selftest_bounded_wait_rejects_bad_arguments_before_launching():
     dummy = ctypes.c_void_p(16)  # never dereferenced: validation fails first
     assert L.bha_selftest_bounded_wait(0, dummy, None) == -1        # limit below range
     assert L.bha_selftest_bounded_wait(5_000_000_000, dummy, None) == -1  # above range
+
+
+def test_header_is_plain_c99_and_declares_every_entry_point():
+    """bha.h compiles as C99 on its own (no C++ or torch types), with the argument types of
+    every entry point as tests/c_header_check.c spells them."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-fsyntax-only",
+                        "-I", os.path.join(root, "include"),
+                        os.path.join(root, "tests", "c_header_check.c")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
