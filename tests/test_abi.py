@@ -153,3 +153,17 @@ def test_header_is_plain_c99_and_declares_every_entry_point():
                         os.path.join(root, "tests", "c_header_check.c")],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_teacher_splits_the_key_range_only_where_it_pays():
+    """The teacher's workspace (fp32 partials of nsplit key ranges; zero when unsplit) follows
+    its cost model: 64 requests x 4 KV heads already fill the GPU, so caches up to 8K tokens
+    run unsplit and a 32K cache splits 4 ways; a few requests with a long cache split so that
+    the key range spreads over the SMs."""
+    T, Hq, d = 64 * 32, 16, 128
+    per_split = T * Hq * (d + 2) * 4
+    for P in (512, 2048, 8192):
+        assert bha.full_prefix_workspace_bytes(64, Hq, 4, d, 32, T, P + 32) == 0
+    assert bha.full_prefix_workspace_bytes(64, Hq, 4, d, 32, T, 32768 + 32) == 4 * per_split
+    # 3 requests x 2 KV heads, 2000-token cache (16 tiles of 128 keys): 4 splits of 4 tiles
+    assert bha.full_prefix_workspace_bytes(3, 8, 2, d, 32, 54, 2000) == 4 * 54 * 8 * (d + 2) * 4
