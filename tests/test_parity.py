@@ -208,6 +208,28 @@ def test_decode_step_ragged_slots_gate_isolated_states():
     assert_close(host64(O), want, TOL_BF16, "O")
 
 
+def test_decode_step_large_queries_mixed_shift_paths():
+    """Queries of some 8-token groups scaled by 4, and of one request by 8 (exact in bf16), so
+    that in those rows max u - min u may reach ~50-100 log2 units: the feature-map warps that
+    hold them take the full max/min pass, the other warps of the same units keep the shift
+    from their first 32 features; ragged blocks, the gate and drawn states; every row checked."""
+    c = inputs.decode_case(R=6, Hq=16, Hkv=4, d=128, F=256, block_lens=[32, 32, 20, 9, 32, 32],
+                           prefix_lens=0, seed=41, dtype="bf16", with_alpha=True)
+    Q = c.Q.copy()
+    lo = c.cu_blk
+    Q[lo[0] + 8:lo[0] + 16] *= 4
+    Q[lo[2]:lo[3]] *= 8
+    Q[lo[4]:lo[4] + 8] *= 4
+    Q[lo[5] + 24:lo[5] + 32] *= 4
+    c.Q = Q
+    S_np, Z_np = inputs.random_states(6, 4, 256, 128, prefix_len=500, seed=9)
+    S, Z = dev(S_np, torch.float32), dev(Z_np, torch.float32)
+    O = run_hybrid(c, S, Z, alpha=c.alpha)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, S_np, Z_np, c.W, c.alpha)
+    assert np.isfinite(host64(O)).all()
+    assert_close(host64(O), want, TOL_BF16, "O")
+
+
 def test_empty_prefix_is_block_softmax():
     c = inputs.decode_case(R=4, Hq=16, Hkv=4, d=128, F=256, block_lens=[32, 5, 32, 1],
                            prefix_lens=0, seed=4, dtype="bf16", with_alpha=True)
