@@ -441,7 +441,9 @@ def bench_decode(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16 in, tf32 state read, fp32 accumulate" if variant == 1 else "f32",
+        "dtype": "bf16",
+        "precision": ("bf16 activations; fp32 states read as tf32 by the tensor cores; fp32 "
+                      "accumulation" if variant == 1 else "bf16 activations; fp32 arithmetic"),
         "data": "synthetic", "config": decode_config(),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
@@ -515,7 +517,8 @@ def bench_commit(args, world, rank, local):
                "l2": f"rotating {NSETS} state sets of ~75 MB each, together larger than the 126 MB L2"}
         print(json.dumps(_line("block-commit tokens/s (128 reqs x 4 KV heads)",
                                R * B * world / (ms_step / 1e3), UNIT, args, world, ms_step, True, cfg,
-                               dtype="bf16 in, fp32 state", kernel_variant=bha.kernel_variant(dims, 2),
+                               dtype="bf16", precision="bf16 activations; fp32 states and accumulation",
+                               kernel_variant=bha.kernel_variant(dims, 2),
                                roofline=_roof(commit_bytes(), ms_step, peaks, src, "commit",
                                               flops=2 * R * HKV * B * (D * (F // 2) + F * D + F),
                                               traffic=profiled_traffic("commit", source_hash("commit_tc.cu"))
@@ -550,7 +553,7 @@ def bench_featuremap(args, world, rank, local):
                            "256, fp32 output", "tokens": R * B, "heads": HQ, "head_dim": D,
                "feature_dim": F, "l2": "2 rotating sets of ~84 MB each, together larger than the 126 MB L2"}
         print(json.dumps(_line("feature-map rows/s", rows * world / (ms_step / 1e3), "rows/s", args,
-                               world, ms_step, True, cfg, dtype="bf16 in, f32 out",
+                               world, ms_step, True, cfg, dtype="bf16", precision="bf16 x and W; fp32 u and phi",
                                roofline=_roof(nbytes, ms_step, peaks, src, "featuremap",
                                               flops=2 * rows * D * (F // 2),
                                               traffic=profiled_traffic("featuremap",
@@ -676,7 +679,7 @@ def bench_cycle(args, world, rank, local):
                "steps_per_block": nsteps, "prefix_mean": float(plen.mean())}
         print(json.dumps(_line("serving-cycle tokens/s per denoise step (6 hybrid layers)",
                                nsteps * R * B * world / (ms_cycle / 1e3), UNIT, args, world,
-                               ms_cycle, True, cfg, dtype="bf16 in, fp32 state",
+                               ms_cycle, True, cfg, dtype="bf16", precision="bf16 activations; fp32 states",
                                roofline=_roof(nbytes, ms_cycle, peaks, src, "block cycle"),
                                committed_tokens_per_s=R * B * world / (ms_cycle / 1e3),
                                gpu_launches=args.steps * (nsteps * layers + layers))), flush=True)
