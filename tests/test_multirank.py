@@ -8,7 +8,6 @@ import datetime
 import importlib.util
 import os
 import socket
-import sys
 
 import pytest
 import torch
