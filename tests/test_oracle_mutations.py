@@ -7,17 +7,17 @@ The slips are the ones the method invites ("Retrofitting Linear Attention into D
 Language Models", §2.2 and §3.1): the sign of the -xW half of phi, one softmax over both
 halves, W transposed, the 1/sqrt(d) temperature dropped or squared, the gate inverted or
 moved to the other branch, a normaliser term dropped, keys and values swapped in the state,
-a commit that overwrites instead of adding, the active block also read through the
-states, a causal mask inside the block, contiguous vs interleaved query-head groups, the
-feature-map head-to-weight map, and the teacher's temperature and key window.
+a commit that overwrites instead of adding, Z as a mean, the active block also read through
+the states, a causal mask inside the block, contiguous vs interleaved query-head groups (in
+the decode and in the teacher), the feature-map head-to-weight map, the slot map and the
+gate of the batched calls, the brute-force prefix sum's kernel, and the teacher's
+temperature and key window.
 """
 import concurrent.futures as cf
 import os
 import shutil
 import subprocess
 import sys
-
-import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 ORACLE_SRC = os.path.join(ROOT, "oracle", "bha_ref.py")
@@ -81,6 +81,24 @@ MUTANTS = [
     ("teacher without 1/sqrt(d)",
      "s = (q @ k.T) / np.sqrt(d)",
      "s = q @ k.T"),
+    ("batched decode ignores the slot map",
+     "if hi == lo:\n            continue\n        slot = r if state_slot is None else int(state_slot[r])",
+     "if hi == lo:\n            continue\n        slot = r"),
+    ("batched commit ignores the slot map",
+     "lo, hi = int(cu_blk[r]), int(cu_blk[r + 1])\n        slot = r if state_slot is None else int(state_slot[r])",
+     "lo, hi = int(cu_blk[r]), int(cu_blk[r + 1])\n        slot = r"),
+    ("batched decode drops the gate",
+     "w = 1.0 if alpha is None else float(gate(alpha[h]))",
+     "w = 1.0"),
+    ("Z as the mean of phi(k) instead of the sum",
+     "return P.T @ V, P.sum(axis=0)",
+     "return P.T @ V, P.mean(axis=0)"),
+    ("brute-force linear kernel halved",
+     "kern = fq @ phi(K_pre[t], W)  # [b]",
+     "kern = 0.5 * (fq @ phi(K_pre[t], W))  # [b]"),
+    ("teacher with interleaved query-head groups",
+     "g = h // G\n            O[lo:hi, h] = softmax_attn_head",
+     "g = h % Hkv\n            O[lo:hi, h] = softmax_attn_head"),
     ("teacher drops the last cached key",
      "softmax_attn_head(Q[lo:hi, h], Kc[r, g, :n], Vc[r, g, :n])",
      "softmax_attn_head(Q[lo:hi, h], Kc[r, g, :n - 1], Vc[r, g, :n - 1])"),
