@@ -15,8 +15,11 @@ shape. The shape is d 128, F 256, 4 query heads per KV head, 32-token blocks, st
 1024-token prefixes and a random gate. It then compares the result with the float64
 oracle. It shows how much of the parity tolerance (max-abs 2e-2, rel-L2 5e-3) the design's
 roundings use by themselves, and which rounding dominates. What is left covers summation
-order, the hardware exp2 approximation, and the states' own rounding when the commit kernel
-builds them (bf16 phi). The model shares no code with the CUDA path.
+order and the hardware exp2 approximation. A second model applies the commit kernel's
+roundings in the same way: phi of the block's keys in fp32, rounded to bf16 for the phi^T V
+product, fp32 accumulation and fp32 read-modify-write of S and Z. It shows what 32
+sequential commits cost the states, and what that costs the decode step. The models share
+no code with the CUDA path.
 """
 import numpy as np
 
@@ -128,3 +131,44 @@ def test_budget_holds_for_large_queries():
     want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, S, Z, c.W, c.alpha)
     max_abs, rel = _err(model_decode(c, S, Z), want)
     assert max_abs <= TOL["max_abs"] and rel <= TOL["rel_l2"], (max_abs, rel)
+
+
+def model_phi(x, W):
+    """phi as the commit kernel forms it: u in fp32, each half's softmax in fp32."""
+    u = f32(x @ W)
+
+    def half(z):
+        e = f32(np.exp(z - z.max(-1, keepdims=True)))
+        return f32(e / f32(e.sum(-1, keepdims=True)))
+
+    return np.concatenate([half(u), half(-u)], -1)
+
+
+def model_commits(Kp, Vp, W, blk=32):
+    """States built by sequential commits of `blk`-token blocks: S += bf16(phi)^T V and
+    Z += sum of bf16(phi), accumulated in fp32 and stored in fp32."""
+    S = np.zeros((2 * W.shape[1], W.shape[0]))
+    Z = np.zeros(2 * W.shape[1])
+    for s0 in range(0, Kp.shape[0], blk):
+        P = bf16(model_phi(Kp[s0:s0 + blk].astype(np.float64), W))
+        S = f32(S + f32(P.T @ Vp[s0:s0 + blk].astype(np.float64)))
+        Z = f32(Z + f32(P.sum(0)))
+    return S, Z
+
+
+def test_commit_roundings_and_the_decode_on_committed_states():
+    """32 commits of 32 tokens: the states stay within half the tolerance of the oracle's
+    one-shot states, and the decode step on them within half the tolerance of the oracle."""
+    c, S, Z = _serving_case()
+    Sm, Zm = np.zeros_like(S), np.zeros_like(Z)
+    for r in range(c.R):
+        lo, hi = c.cu_pre[r], c.cu_pre[r + 1]
+        for g in range(c.Hkv):
+            Sm[r, g], Zm[r, g] = model_commits(c.K_pre[lo:hi, g], c.V_pre[lo:hi, g],
+                                               c.W[g].astype(np.float64))
+    for got, ref_state in ((Sm, S), (Zm, Z)):
+        max_abs, rel = _err(got, ref_state)
+        assert max_abs <= 0.5 * TOL["max_abs"] and rel <= 0.5 * TOL["rel_l2"], (max_abs, rel)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, S, Z, c.W, c.alpha)
+    max_abs, rel = _err(model_decode(c, Sm, Zm), want)
+    assert max_abs <= 0.5 * TOL["max_abs"] and rel <= 0.5 * TOL["rel_l2"], (max_abs, rel)
