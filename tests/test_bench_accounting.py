@@ -1,0 +1,45 @@
+"""The roofline numerators bench.py reports: algorithmic bytes and FLOPs per launch, checked on
+the CPU against the figures stated for each workload, and against the byte sizes of the
+tensors each call reads and writes once (numel x element size)."""
+import importlib.util
+import os
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_accounting", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_decode_step_bytes_and_flops():
+    b = _bench()
+    R, Hq, Hkv, d, F, B = 128, 16, 4, 128, 256, 32
+    T = R * B
+    tensors = {  # numel x bytes, each read or written once per step
+        "S": R * Hkv * F * d * 4, "Z": R * Hkv * F * 4, "Q": T * Hq * d * 2, "K": T * Hkv * d * 2,
+        "V": T * Hkv * d * 2, "O": T * Hq * d * 2, "W": Hkv * d * (F // 2) * 2,
+    }
+    assert tensors == {"S": 67_108_864, "Z": 524_288, "Q": 16_777_216, "K": 4_194_304,
+                       "V": 4_194_304, "O": 16_777_216, "W": 131_072}
+    assert b.step_bytes() == sum(tensors.values()) == 109_707_264
+    # per (request, query head): q.W 1,048,576 + q.k 262,144 + P.V 262,144 + phi.S 2,097,152
+    # + phi.Z 16,384 FLOPs over the block's 32 queries
+    assert b.step_flops() == R * Hq * 3_686_400 == 7_549_747_200
+
+
+def test_commit_bytes():
+    b = _bench()
+    R, Hkv, d, F, B = 128, 4, 128, 256, 32
+    rmw = 2 * (R * Hkv * F * d * 4 + R * Hkv * F * 4)
+    kv = 2 * R * B * Hkv * d * 2
+    assert b.commit_bytes() == rmw + kv + Hkv * d * (F // 2) * 2 == 143_785_984
+
+
+def test_teacher_bytes_over_the_prefix_sweep():
+    b = _bench()
+    for P, want in ((512, 88_080_384), (2048, 289_406_976), (8192, 1_094_713_344),
+                    (32768, 4_315_938_816)):
+        assert b.teacher_bytes(64, 16, 4, 128, 32, P) == 16_777_216 + 131_072 * (P + 32) == want
