@@ -14,12 +14,14 @@
 //   dZ    = column sums of the bf16 phi over each request's tokens (CUDA cores)
 //   dS^T  = V_r^T phi_r           bf16 MMA per request, M 128 (d), N 256 (F), K 32 (tokens)
 //                                 into one of two TMEM buffers
-//   S += dS, Z += dZ               fp32 read-modify-write by 8 warps: TMEM lane = d, so each
-//                                 warp instruction reads or writes one whole 128-byte line
-//                                 of a row of S, 64 rows per thread in flight at a time;
-//                                 the other buffer's MMA overlaps it.
-// Computing dS transposed (lanes = d) is what makes the state update coalesced without
-// staging it through shared memory.
+//   S += dS, Z += dZ               TMA bulk reduce-add: each of 8 warps copies 16 columns of
+//                                 dS^T at a time from TMEM (its lane quarter = 32 values of d)
+//                                 into a 2 KiB shared tile [16 rows of F][32 d] and hands it
+//                                 to the tensor memory accelerator, which adds it into S in
+//                                 L2; Z by reducing atomic adds.  No thread waits on a load of
+//                                 S, and the other dS buffer's MMA overlaps the update.
+// Computing dS transposed (lanes = d) is what lets each warp write whole 128-byte rows of its
+// shared tile, one per instruction, without bank conflicts.
 //
 // Roles (320 threads): warp 0 TMA producer (K, V, W), warp 1 TMEM owner and MMA issuer,
 // warps 2-9 feature map, dZ and the state update.  Every wait is bounded; on expiry the CTA
@@ -45,6 +47,7 @@ constexpr uint32_t kKBytes = kM * kD * 2;        // 32 KiB: [d half][128 rows][1
 constexpr uint32_t kWBytes = kD * kFh * 2;       // 32 KiB: [f half][128 rows of d][128 B]
 constexpr uint32_t kVReqBytes = kBlk * kD * 2;   // 8 KiB per request: [d half][32 rows][128 B]
 constexpr uint32_t kPhiReqBytes = kBlk * kF * 2; // 16 KiB per request: [f quarter][32 rows][128 B]
+constexpr int kRedRows = 16;                      // F rows per reduce-add tile
 
 constexpr uint32_t kColU = 0;     // u (128 columns), inside dS buffer 0
 constexpr uint32_t kColD0 = 0;    // dS^T buffers: 256 columns each
@@ -60,6 +63,7 @@ struct __align__(1024) Smem {
   uint8_t v[kReq][kVReqBytes];
   uint8_t phi[kReq][kPhiReqBytes];
   float dz[kReq][kF];
+  float red[8][2][kRedRows * 32];  // per update warp, double-buffered: [16 rows of F][32 d]
   uint64_t k_full, k_empty, v_full, v_empty, w_full, u_full, phi_ready;
   uint64_t d_full[2], d_empty[2], drain;
   uint32_t tmem_base;
@@ -120,6 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
     tc::prefetch_tensormap(&p.tm_k);
     tc::prefetch_tensormap(&p.tm_v);
     tc::prefetch_tensormap(&p.tm_w);
+    tc::prefetch_tensormap(&p.tm_s);
   }
   if (warp == 1) {
     tc::tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -253,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
     const int tid = sw * 32 + lane;   // 0..255
     const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
     const float log2e = 1.4426950408889634f;
-    int k = 0, rc = 0;
+    int k = 0, rc = 0, nred = 0;
     // A failed wait does not leave the loop at once: these 256 threads meet at a named barrier
     // each unit, so all of them reach it and leave together, decided by the reducing barrier.
     // Work done after a failed wait goes no further than shared memory (S and Z are not
@@ -348,8 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.phi_ready);
 
-      // ---- state update per request: S[f][d] += dS^T[d][f], Z[f] += dZ[f]
-      const int d = row;  // TMEM lane = d
+      // ---- state update per request: S[f][d] += dS^T[d][f] by tiled reduce-add, Z[f] += dZ[f]
       for (int j = 0; j < kReq; ++j) {
         if (rq[j].n == 0) continue;
         const int b = rc & 1;
@@ -357,31 +361,37 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
         good = __all_sync(0xffffffffu, tc::mbar_wait(&sm.d_full[b], (rc >> 1) & 1, abort_flag, lim));
         if (!good) break;
         tc::tc_fence_after();
-        float* Sg = p.S + ((size_t)rq[j].slot * p.Hkv + g) * kF * kD;
+        const int srow0 = (rq[j].slot * p.Hkv + g) * kF + half * kFh;
         const uint32_t col0 = (b ? kColD1 : kColD0) + half * kFh;
-        // 64 state values per thread in flight at a time (64 KiB per CTA): the update is bound
-        // by the round trips of these loads, so each round moves as much as registers allow
 #pragma unroll 1
-        for (int fc = 0; fc < kFh / 64; ++fc) {
-          float dv[64], sv[64];
-          const int f0 = half * kFh + fc * 64;
-#pragma unroll
-          for (int i = 0; i < 64; ++i) sv[i] = Sg[(size_t)(f0 + i) * kD + d];
-          tc::tmem_ld32(tl + col0 + fc * 64, *reinterpret_cast<float(*)[32]>(dv));
-          tc::tmem_ld32(tl + col0 + fc * 64 + 32, *reinterpret_cast<float(*)[32]>(dv + 32));
+        for (int fc = 0; fc < kFh / kRedRows; ++fc, ++nred) {
+          float dv[kRedRows];
+          tc::tmem_ld16(tl + col0 + fc * kRedRows, dv);
+          // the tile's previous reduce (two tiles back) has read it
+          if (lane == 0 && nred >= 2) tc::bulk_wait_read<1>();
+          __syncwarp();
           tc::tmem_wait_ld();
+          float* tile = sm.red[sw][nred & 1];
 #pragma unroll
-          for (int i = 0; i < 64; ++i) Sg[(size_t)(f0 + i) * kD + d] = sv[i] + dv[i];
+          for (int i = 0; i < kRedRows; ++i) tile[i * 32 + lane] = dv[i];
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tc::tma_reduce_add_2d(&p.tm_s, tile, wq * 32, srow0 + fc * kRedRows);
+            tc::bulk_commit();
+          }
         }
-        float* Zg = p.Z + ((size_t)rq[j].slot * p.Hkv + g) * kF;
-        Zg[tid] += sm.dz[j][tid];
+        // every column of this dS buffer has been read: the next request's MMA may reuse it
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&sm.d_empty[b]);
+        atomicAdd(p.Z + ((size_t)rq[j].slot * p.Hkv + g) * kF + tid, sm.dz[j][tid]);
         ++rc;
       }
       ++k;
     }
+    // every reduce this warp started has completed (its shared tile read, its adds performed)
+    if (lane == 0) tc::bulk_wait_all();
   }
 
   tc::tc_fence_before();
@@ -413,6 +423,13 @@ cudaError_t launch_commit_tc(const CommitArgs& a, cudaStream_t st) {
     const uint64_t strides[1] = {kFh * 2};
     const uint32_t box[2] = {64, kD};
     if (!make_tensor_map(&p.tm_w, false, 2, a.W, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
+  }
+  {
+    // reduce-add target: S as rows of d fp32 values, 16 x 32 boxes (one warp's tile)
+    const uint64_t dims[2] = {kD, (uint64_t)a.num_slots * a.Hkv * kF};
+    const uint64_t strides[1] = {kD * 4};
+    const uint32_t box[2] = {32, kRedRows};
+    if (!make_tensor_map(&p.tm_s, true, 2, a.S, dims, strides, box, kTmaNone)) return cudaErrorInvalidValue;
   }
   p.cu_blk = a.cu_blk;
   p.state_slot = a.state_slot;

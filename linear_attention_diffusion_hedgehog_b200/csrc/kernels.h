@@ -59,13 +59,13 @@ struct TcHybridParams {
   const float* alpha;
   __nv_bfloat16* O;
   int32_t* dev_err;
-  int R, Hq, Hkv, T, Bmax, num_slots;
+  int r0, R, Hq, Hkv, T, Bmax, num_slots;  // requests r0 .. r0 + R - 1 of the call
   long long wait_limit;  // SM cycles a bounded wait may spin before giving up
 };
 
 // Parameters of the tensor-core block-commit kernel (commit_tc.cu).
 struct TcCommitParams {
-  CUtensorMap tm_k, tm_v, tm_w;
+  CUtensorMap tm_k, tm_v, tm_w, tm_s;  // tm_s: S as [rows of F][d] fp32, the reduce-add target
   const int32_t* cu_blk;
   const int32_t* state_slot;
   float* S;
