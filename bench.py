@@ -2,9 +2,9 @@
 """Throughput of the block-hybrid attention decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode|commit|sweep|cycle]
+                    [--workload all|decode|commit|featuremap|per_qhead|sweep|cycle]
 
-Default workload ("decode"): one denoising step of one block-hybrid layer for 128 requests
+Headline workload ("decode"): one denoising step of one block-hybrid layer for 128 requests
 with 32-token active blocks, 16 query / 4 KV heads, head dim 128, feature dim 256 (W is
 128 x 128 per KV head), each request's 1024-token prefix held only as fp32 states
 S [4, 256, 128] and Z [4, 256]; bf16 activations ~ N(0, 1), W ~ N(0, 1/128), states built
@@ -18,10 +18,13 @@ bracketed by a barrier and a synchronize, timed with CUDA events on the launchin
 max over ranks.  L2 is defeated by rotating 4 independent input/state sets (4 x 110 MB
 against a 126 MB L2).  Multi-GPU runs are independent replicas (no collective on the path).
 
-Other workloads print their own JSON line: "commit" (the block-commit update for 128
-requests x 4 KV heads), "sweep" (the decode step vs the in-run full-prefix softmax teacher
-at 64 requests over prefixes of 512..32768 tokens) and "cycle" (a ragged serving mix of 128
-requests, 6 hybrid layers, 8 denoising steps then a commit, as one CUDA graph).
+The default run ("all") adds, under "workloads", one record per other workload, each timed
+the same way with its own roofline: the gated decode step, the block commit (128 requests x
+4 KV heads), the standalone feature map, the per-query-head layout (16 state heads), the prefix sweep (decode step on states committed
+from each prefix vs the in-run softmax teacher over the same cache, 64 requests, prefixes
+512..32768, with the teacher's linear fit) and the serving cycle (ragged mix of 128 requests,
+6 layers, 8 denoising steps then a commit, as one CUDA graph), plus the state-vs-KV-cache
+capacity figures.  --workload X runs one of them alone.
 """
 from __future__ import annotations
 
@@ -366,12 +369,97 @@ def decode_config():
                   f"than the 126 MB L2"}
 
 
-def bench_decode(args, world, rank, local):
+def _roof(nbytes, ms, peaks, peak_src, kernel, flops=None, traffic=None):
+    achieved = nbytes / (ms / 1e3) / 1e9
+    r = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+         "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+         "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": nbytes,
+         "kernel": kernel}
+    if flops is not None:
+        r["flops_per_launch"] = flops
+    return r
+
+
+def _record(metric, value, unit, steps, ms_step, config, **extra):
+    d = {"metric": metric, "value": value, "unit": unit, "steps": steps, "ms_per_step": ms_step,
+         "higher_is_better": True, "config": config}
+    d.update(extra)
+    return d
+
+
+def _traffic_for(kernel_key, variant, src_file):
+    return profiled_traffic(kernel_key, source_hash(src_file)) if variant == 1 else None
+
+
+def e2e_pipelined(sets, cu, W, steps, world, stream, alpha=None):
+    """Decode steps end to end through the public API with pinned host buffers: every step
+    copies its Q, K, V host -> device, runs the step and copies O device -> host.  Three
+    streams pipeline consecutive steps (step i+1's inputs go up while step i computes and step
+    i-1's output comes down, so both PCIe directions run at once), with two device buffer sets
+    and events ordering each reuse.  Returns (ms, h2d bytes, d2h bytes) per the whole run."""
+    from linear_attention_diffusion_hedgehog_b200 import bha
+
+    hsets = [{k: sets[i][k].cpu().pin_memory() for k in ("Q", "K", "V")} for i in range(len(sets))]
+    dbuf = [{k: torch.empty_like(sets[0][k]) for k in ("Q", "K", "V", "O")} for _ in range(2)]
+    hout = [torch.empty(sets[0]["O"].shape, dtype=sets[0]["O"].dtype).pin_memory() for _ in range(2)]
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def step(i):
+        b, s, h = i % 2, sets[i % len(sets)], hsets[i % len(hsets)]
+        with torch.cuda.stream(up):
+            if i >= 2:
+                up.wait_event(ev_done[b])      # step i-2 has read this buffer set
+            for k in ("Q", "K", "V"):
+                dbuf[b][k].copy_(h[k], non_blocking=True)
+            ev_in[b].record(up)
+        stream.wait_event(ev_in[b])
+        if i >= 2:
+            stream.wait_event(ev_out[b])       # step i-2's output has left this buffer
+        bha.hybrid_attn(cu, dbuf[b]["Q"], dbuf[b]["K"], dbuf[b]["V"], s["S"], s["Z"], W,
+                        max_block=B, alpha=alpha, out=dbuf[b]["O"], stream=stream)
+        ev_done[b].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_done[b])
+            hout[b].copy_(dbuf[b]["O"], non_blocking=True)
+            ev_out[b].record(down)
+
+    for i in range(4):
+        step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(up)
+    for i in range(steps):
+        step(i)
+    down.wait_stream(stream)
+    e1.record(down)
+    torch.cuda.synchronize()
+    barrier(world)
+    h2d = sum(hsets[0][k].numel() * hsets[0][k].element_size() for k in ("Q", "K", "V"))
+    d2h = hout[0].numel() * hout[0].element_size()
+    return e0.elapsed_time(e1), h2d, d2h
+
+
+def capacity_record(S, Z, Hkv=HKV, d=D, act_bytes=2):
+    """State bytes of one request in one hybrid layer, from the state buffers themselves,
+    against the KV cache the softmax teacher keeps for the same request (K and V per token)."""
+    state = S[0].numel() * S.element_size() + Z[0].numel() * Z.element_size()
+    kv_per_token = 2 * Hkv * d * act_bytes
+    rec = {"state_bytes_per_request_layer": state, "kv_bytes_per_token_layer": kv_per_token,
+           "break_even_prefix_tokens": state / kv_per_token}
+    for P in (1024, 4096, 32768):
+        rec[f"kv_over_state_at_{P}"] = P * kv_per_token / state
+    return rec
+
+
+def bench_decode(args, world, rank, local, gen):
+    """The headline: one decode step of one layer, 128 requests (see the module docstring)."""
     from linear_attention_diffusion_hedgehog_b200 import bha
 
     peaks, peak_src = load_peaks()
-    gen = torch.Generator(device="cuda")
-    gen.manual_seed(1234 + rank)
     W, cu, sets = make_decode_sets(gen)
     stream = torch.cuda.Stream()
     dims = bha.make_dims(R, HQ, HKV, D, F, B, R * B, R, torch.bfloat16)
@@ -394,49 +482,37 @@ def bench_decode(args, world, rank, local):
     step_ms = ms / args.steps
     value = whole_job_rate(R * B, args.steps, ms, world)
 
-    # end to end through the public API: pinned host Q/K/V in, O back to pinned host
     e2e_steps = min(args.steps, 200)
-    hsets = [{k: sets[i][k].cpu().pin_memory() for k in ("Q", "K", "V")} for i in range(NSETS)]
-    hout = torch.empty(sets[0]["O"].shape, dtype=torch.bfloat16).pin_memory()
-    dQ = torch.empty_like(sets[0]["Q"])
-    dK = torch.empty_like(sets[0]["K"])
-    dV = torch.empty_like(sets[0]["V"])
-    h2d = sum(hsets[0][k].numel() * 2 for k in ("Q", "K", "V"))
-    d2h = hout.numel() * 2
-
-    def e2e_step(i):
-        s, h = sets[i % NSETS], hsets[i % NSETS]
-        with torch.cuda.stream(stream):
-            dQ.copy_(h["Q"], non_blocking=True)
-            dK.copy_(h["K"], non_blocking=True)
-            dV.copy_(h["V"], non_blocking=True)
-            bha.hybrid_attn(cu, dQ, dK, dV, s["S"], s["Z"], W, max_block=B, out=s["O"],
-                            stream=stream)
-            hout.copy_(s["O"], non_blocking=True)
-
-    for i in range(3):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e_ms, h2d, d2h = e2e_pipelined(sets, cu, W, e2e_steps, world, stream)
+    e2e_ms = max_over_ranks(e2e_ms, world)
     e2e_value = whole_job_rate(R * B, e2e_steps, e2e_ms, world)
 
+    # the same step with the sigmoid gate on (alpha ~ N(0, 1) per query head)
+    alpha = torch.randn((HQ,), generator=gen, device="cuda")
+    gsteps = min(args.steps, 2000)
+
+    def gstep(i):
+        s = sets[i % NSETS]
+        bha.hybrid_attn(cu, s["Q"], s["K"], s["V"], s["S"], s["Z"], W, max_block=B, alpha=alpha,
+                        out=s["O"], stream=stream)
+
+    g_ms = max_over_ranks(time_graphed(gstep, gsteps, args.warmup, world, stream), world) / gsteps
+    src = "hybrid_tc.cu" if variant == 1 else "simt.cu"
+    nbytes = step_bytes() + HQ * 4
+    gated = _record("hybrid-attn tokens/s per denoise step, gated merge (alpha ~ N(0,1))",
+                    whole_job_rate(R * B, gsteps, g_ms * gsteps, world), UNIT, gsteps, g_ms,
+                    dict(decode_config(), gate="alpha ~ N(0, 1) per query head"),
+                    roofline=_roof(nbytes, g_ms, peaks, peak_src, "hybrid tensor-core" if variant == 1
+                                   else "hybrid generic", flops=step_flops()),
+                    gpu_launches=gsteps)
+    capacity = capacity_record(sets[0]["S"], sets[0]["Z"])
+    del sets
+    torch.cuda.empty_cache()
     if rank != 0:
-        return
+        return None
     nbytes = step_bytes()
     achieved = nbytes / (step_ms / 1e3) / 1e9
     peak = peaks["hbm_gbs"]
-    src = source_hash("hybrid_tc.cu") if variant == 1 and os.path.exists(
-        os.path.join(ROOT, "linear_attention_diffusion_hedgehog_b200", "csrc", "hybrid_tc.cu")) \
-        else source_hash("simt.cu")
-    traffic = profiled_traffic("hybrid_decode", src)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
@@ -446,15 +522,18 @@ def bench_decode(args, world, rank, local):
                       "accumulation" if variant == 1 else "bf16 activations; fp32 arithmetic"),
         "data": "synthetic", "config": decode_config(),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic,
+                     "frac": achieved / peak, "traffic": _traffic_for("hybrid_decode", variant, src),
                      "peak_source": f"{peak_src} hbm_gbs",
                      "algorithmic_bytes_per_launch": nbytes, "flops_per_launch": step_flops(),
                      "kernel": "hybrid tensor-core" if variant == 1 else "hybrid generic"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "pipelining": "3 streams: next step's H2D and previous step's D2H overlap this "
+                              "step's kernel"},
         "gpu_launches": args.steps,
         "clocks": clocks,
         "kernel_variant": variant,
+        "workloads": {"decode_gated": gated, "capacity": capacity},
     }
     if world == 1 and not args.no_cpu_baseline:
         n, el, cores = cpu_oracle_decode(budget_s=12.0)
@@ -463,30 +542,10 @@ def bench_decode(args, world, rank, local):
                                 "sample": f"{n} whole requests of the decode step (16 query heads x "
                                           f"32 tokens, states given; one request repeated), "
                                           f"{el:.1f} s"}
-    print(json.dumps(line), flush=True)
+    return line
 
 
-# ------------------------------------------------------------------ other workloads
-def _line(metric, value, unit, args, world, ms_step, higher, config, **extra):
-    d = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": higher,
-         "scaling": "weak", "vs_baseline": None, "data": "synthetic", "config": config}
-    d.update(extra)
-    return d
-
-
-def _roof(nbytes, ms, peaks, peak_src, kernel, flops=None, traffic=None):
-    achieved = nbytes / (ms / 1e3) / 1e9
-    r = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-         "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-         "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": nbytes,
-         "kernel": kernel}
-    if flops is not None:
-        r["flops_per_launch"] = flops
-    return r
-
-
-def bench_commit(args, world, rank, local):
+def bench_commit(args, world, rank, local, steps):
     """Block commit for 128 requests x 4 KV heads (d 128, F 256, 32-token blocks): S and Z
     updated in place; 4 rotating state sets (75 MB each) keep L2 from holding them."""
     from linear_attention_diffusion_hedgehog_b200 import bha
@@ -503,30 +562,30 @@ def bench_commit(args, world, rank, local):
                  Z=torch.rand((R, HKV, F), generator=gen, device=dev) * 8) for _ in range(NSETS)]
     stream = torch.cuda.Stream()
     dims = bha.make_dims(R, HKV, HKV, D, F, B, R * B, R, bf)
+    variant = bha.kernel_variant(dims, 2)
 
     def step(i):
         s = sets[i % NSETS]
         bha.commit_block(cu, s["K"], s["V"], W, s["S"], s["Z"], max_block=B, stream=stream)
 
-    ms = max_over_ranks(time_graphed(step, args.steps, args.warmup, world, stream), world)
-    if rank == 0:
-        ms_step = ms / args.steps
-        cfg = {"workload": "block commit: fold a 32-token block into S/Z for 128 requests x 4 KV "
-                           "heads, head dim 128, feature dim 256", "requests": R, "kv_heads": HKV,
-               "head_dim": D, "feature_dim": F, "block": B,
-               "l2": f"rotating {NSETS} state sets of ~75 MB each, together larger than the 126 MB L2"}
-        print(json.dumps(_line("block-commit tokens/s (128 reqs x 4 KV heads)",
-                               R * B * world / (ms_step / 1e3), UNIT, args, world, ms_step, True, cfg,
-                               dtype="bf16", precision="bf16 activations; fp32 states and accumulation",
-                               kernel_variant=bha.kernel_variant(dims, 2),
-                               roofline=_roof(commit_bytes(), ms_step, peaks, src, "commit",
-                                              flops=2 * R * HKV * B * (D * (F // 2) + F * D + F),
-                                              traffic=profiled_traffic("commit", source_hash("commit_tc.cu"))
-                                              if bha.kernel_variant(dims, 2) == 1 else None),
-                               gpu_launches=args.steps)), flush=True)
+    ms = max_over_ranks(time_graphed(step, steps, args.warmup, world, stream), world)
+    del sets
+    torch.cuda.empty_cache()
+    ms_step = ms / steps
+    cfg = {"workload": "block commit: fold a 32-token block into S/Z for 128 requests x 4 KV "
+                       "heads, head dim 128, feature dim 256", "requests": R, "kv_heads": HKV,
+           "head_dim": D, "feature_dim": F, "block": B,
+           "l2": f"rotating {NSETS} state sets of ~75 MB each, together larger than the 126 MB L2"}
+    return _record("block-commit tokens/s (128 reqs x 4 KV heads)", whole_job_rate(R * B, steps, ms, world),
+                   UNIT, steps, ms_step, cfg, dtype="bf16",
+                   precision="bf16 activations; fp32 states and accumulation", kernel_variant=variant,
+                   roofline=_roof(commit_bytes(), ms_step, peaks, src, "commit",
+                                  flops=2 * R * HKV * B * (D * (F // 2) + F * D + F),
+                                  traffic=_traffic_for("commit", variant, "commit_tc.cu")),
+                   gpu_launches=steps)
 
 
-def bench_featuremap(args, world, rank, local):
+def bench_featuremap(args, world, rank, local, steps):
     """Standalone feature map phi(x) on the decode step's queries: x [4096, 16, 128] bf16 ->
     phi [4096, 16, 256] fp32, 4 KV-head weight matrices; 2 rotating sets (84 MB each)."""
     from linear_attention_diffusion_hedgehog_b200 import bha
@@ -544,27 +603,38 @@ def bench_featuremap(args, world, rank, local):
         s = sets[i % 2]
         bha.featuremap(s["x"], W, out=s["o"], stream=stream)
 
-    ms = max_over_ranks(time_graphed(step, args.steps, args.warmup, world, stream), world)
-    if rank == 0:
-        ms_step = ms / args.steps
-        rows = R * B * HQ
-        nbytes = rows * D * 2 + rows * F * 4 + HKV * D * (F // 2) * 2
-        cfg = {"workload": "feature map phi(x) of 4096 tokens x 16 heads, head dim 128, feature dim "
-                           "256, fp32 output", "tokens": R * B, "heads": HQ, "head_dim": D,
-               "feature_dim": F, "l2": "2 rotating sets of ~84 MB each, together larger than the 126 MB L2"}
-        print(json.dumps(_line("feature-map rows/s", rows * world / (ms_step / 1e3), "rows/s", args,
-                               world, ms_step, True, cfg, dtype="bf16", precision="bf16 x and W; fp32 u and phi",
-                               roofline=_roof(nbytes, ms_step, peaks, src, "featuremap",
-                                              flops=2 * rows * D * (F // 2),
-                                              traffic=profiled_traffic("featuremap",
-                                                                       source_hash("featuremap_tc.cu"))),
-                               gpu_launches=args.steps)), flush=True)
+    ms = max_over_ranks(time_graphed(step, steps, args.warmup, world, stream), world)
+    del sets
+    torch.cuda.empty_cache()
+    ms_step = ms / steps
+    rows = R * B * HQ
+    nbytes = rows * D * 2 + rows * F * 4 + HKV * D * (F // 2) * 2
+    cfg = {"workload": "feature map phi(x) of 4096 tokens x 16 heads, head dim 128, feature dim "
+                       "256, fp32 output", "tokens": R * B, "heads": HQ, "head_dim": D,
+           "feature_dim": F, "l2": "2 rotating sets of ~84 MB each, together larger than the 126 MB L2"}
+    return _record("feature-map rows/s", whole_job_rate(rows, steps, ms, world), "rows/s", steps,
+                   ms_step, cfg, dtype="bf16", precision="bf16 x and W; fp32 u and phi",
+                   roofline=_roof(nbytes, ms_step, peaks, src, "featuremap", flops=2 * rows * D * (F // 2),
+                                  traffic=_traffic_for("featuremap", 1, "featuremap_tc.cu")),
+                   gpu_launches=steps)
 
 
-def bench_sweep(args, world, rank, local):
+def linear_fit(xs, ys):
+    """Least-squares y = a + b x and its coefficient of determination R^2."""
+    xs, ys = np.asarray(xs, np.float64), np.asarray(ys, np.float64)
+    b, a = np.polyfit(xs, ys, 1)
+    pred = a + b * xs
+    ss_res = float(((ys - pred) ** 2).sum())
+    ss_tot = float(((ys - ys.mean()) ** 2).sum())
+    return float(a), float(b), 1.0 - ss_res / ss_tot if ss_tot > 0 else 1.0
+
+
+def bench_sweep(args, world, rank, local, steps):
     """Decode step vs the full-prefix softmax teacher at 64 requests (16 query / 4 KV heads,
-    head dim 128, 32-token blocks) over prefixes of 512 .. 32768 tokens.  The hybrid reads only
-    the fixed-size states; the teacher reads a bf16 KV cache of prefix + block tokens."""
+    head dim 128, 32-token blocks) over prefixes of 512 .. 32768 tokens.  At each prefix length
+    one KV cache of prefix + block tokens is drawn; the hybrid's states are committed from that
+    cache's prefix tokens (32 at a time, through the library) and the block's own K/V are the
+    cache's last 32 rows, so both kernels see the same request; each is timed at that prefix."""
     from linear_attention_diffusion_hedgehog_b200 import bha
 
     peaks, src = load_peaks()
@@ -572,58 +642,72 @@ def bench_sweep(args, world, rank, local):
     Rs = 64
     gen = torch.Generator(device="cuda")
     gen.manual_seed(5 + rank)
-    W, cu, hsets = make_decode_sets(gen, nsets=NSETS, R=Rs, prefix=0, states_from_commits=False)
-    for s in hsets:
-        s["S"].normal_(generator=gen)
-        s["Z"].uniform_(0.5, 1.5, generator=gen)
+    W = (torch.randn((HKV, D, F // 2), generator=gen, device=dev) / D ** 0.5).to(bf)
+    cu = torch.arange(0, (Rs + 1) * B, B, dtype=torch.int32, device=dev)
     stream = torch.cuda.Stream()
-    steps = args.steps
-
-    def hstep(i):
-        s = hsets[i % NSETS]
-        bha.hybrid_attn(cu, s["Q"], s["K"], s["V"], s["S"], s["Z"], W, max_block=B, out=s["O"],
-                        stream=stream)
-
-    h_ms = max_over_ranks(time_graphed(hstep, steps, args.warmup, world, stream), world) / steps
     out = []
     for P in (512, 2048, 8192, 32768):
         L = P + B
-        cap = L
-        nsets = max(1, min(NSETS, int(np.ceil(400e6 / (Rs * HKV * L * D * 2 * 2)))))
-        tsets = []
-        for _ in range(nsets):
-            Kc = torch.randn((Rs, HKV, cap, D), generator=gen, device=dev).to(bf)
-            Vc = torch.randn((Rs, HKV, cap, D), generator=gen, device=dev).to(bf)
-            tsets.append(dict(Kc=Kc, Vc=Vc, Q=hsets[0]["Q"], O=torch.empty_like(hsets[0]["O"])))
+        Kc = torch.randn((Rs, HKV, L, D), generator=gen, device=dev).to(bf)
+        Vc = torch.randn((Rs, HKV, L, D), generator=gen, device=dev).to(bf)
+        S = torch.zeros((Rs, HKV, F, D), device=dev)
+        Z = torch.zeros((Rs, HKV, F), device=dev)
+        for j in range(0, P, B):
+            bha.commit_block(cu, Kc[:, :, j:j + B].transpose(1, 2).reshape(Rs * B, HKV, D).contiguous(),
+                             Vc[:, :, j:j + B].transpose(1, 2).reshape(Rs * B, HKV, D).contiguous(),
+                             W, S, Z, max_block=B)
+        Kb = Kc[:, :, P:L].transpose(1, 2).reshape(Rs * B, HKV, D).contiguous()
+        Vb = Vc[:, :, P:L].transpose(1, 2).reshape(Rs * B, HKV, D).contiguous()
+        hsets = [dict(Q=torch.randn((Rs * B, HQ, D), generator=gen, device=dev).to(bf), K=Kb.clone(),
+                      V=Vb.clone(), S=S.clone(), Z=Z.clone(),
+                      O=torch.empty((Rs * B, HQ, D), device=dev, dtype=bf)) for _ in range(NSETS)]
+
+        def hstep(i):
+            s = hsets[i % NSETS]
+            bha.hybrid_attn(cu, s["Q"], s["K"], s["V"], s["S"], s["Z"], W, max_block=B, out=s["O"],
+                            stream=stream)
+
+        h_ms = max_over_ranks(time_graphed(hstep, steps, args.warmup, world, stream), world) / steps
         kv_len = torch.full((Rs,), L, dtype=torch.int32, device=dev)
-        ws_bytes = bha.full_prefix_workspace_bytes(Rs, HQ, HKV, D, B, Rs * B, cap)
+        ws_bytes = bha.full_prefix_workspace_bytes(Rs, HQ, HKV, D, B, Rs * B, L)
         ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        nsets = max(1, min(NSETS, int(np.ceil(400e6 / (Rs * HKV * L * D * 2 * 2)))))
+        tsets = [dict(Kc=Kc, Vc=Vc)] + [dict(Kc=Kc.clone(), Vc=Vc.clone()) for _ in range(nsets - 1)]
+        tO = torch.empty((Rs * B, HQ, D), device=dev, dtype=bf)
 
         def tstep(i):
             s = tsets[i % nsets]
-            bha.full_prefix_attn(cu, kv_len, s["Q"], s["Kc"], s["Vc"], max_block=B, workspace=ws,
-                                 out=s["O"], stream=stream)
+            bha.full_prefix_attn(cu, kv_len, hsets[i % NSETS]["Q"], s["Kc"], s["Vc"], max_block=B,
+                                 workspace=ws, out=tO, stream=stream)
 
         tsteps = max(3, min(steps, int(2e5 // max(P, 1))))
         t_ms = max_over_ranks(time_graphed(tstep, tsteps, args.warmup, world, stream), world) / tsteps
-        del tsets
+        del tsets, hsets, Kc, Vc, S, Z
         torch.cuda.empty_cache()
         hb = step_bytes(R=Rs)
         tb = teacher_bytes(Rs, HQ, HKV, D, B, P)
         out.append({"prefix": P, "hybrid_ms": h_ms, "teacher_ms": t_ms, "speedup": t_ms / h_ms,
                     "hybrid_hbm_frac": hb / (h_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
                     "teacher_hbm_frac": tb / (t_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-                    "teacher_steps": tsteps})
-    if rank == 0:
-        cfg = {"workload": "hybrid decode step (states only) vs full-prefix softmax teacher, 64 "
-                           "requests, 16 query / 4 KV heads, head dim 128, 32-token blocks",
-               "requests": Rs, "prefixes": [o["prefix"] for o in out]}
-        print(json.dumps(_line("hybrid vs teacher per-block latency over prefix length",
-                               out[-1]["speedup"], "x (teacher/hybrid at 32K prefix)", args, world,
-                               h_ms, True, cfg, dtype="bf16", sweep=out)), flush=True)
+                    "hybrid_steps": steps, "teacher_steps": tsteps})
+    hs = [o["hybrid_ms"] for o in out]
+    a, b, r2 = linear_fit([o["prefix"] for o in out], [o["teacher_ms"] for o in out])
+    cfg = {"workload": "hybrid decode step (states committed from each prefix) vs full-prefix softmax "
+                       "teacher over the same cache, 64 requests, 16 query / 4 KV heads, head dim 128, "
+                       "32-token blocks", "requests": Rs, "prefixes": [o["prefix"] for o in out],
+           "l2": "hybrid: 4 rotating state sets (55 MB each); teacher: caches of 88 MB to 4.3 GB, "
+                 "rotated up to 400 MB"}
+    return _record("hybrid vs teacher per-block latency over prefix length", out[-1]["speedup"],
+                   "x (teacher/hybrid at 32K prefix)", steps, float(np.mean(hs)), cfg, dtype="bf16",
+                   sweep=out,
+                   hybrid_spread=(max(hs) - min(hs)) / float(np.mean(hs)),
+                   teacher_fit={"a_ms": a, "b_ms_per_prefix_token": b, "r2": r2},
+                   roofline=_roof(step_bytes(R=Rs), float(np.mean(hs)), peaks, src,
+                                  "hybrid tensor-core (64 requests, mean over the prefixes)"),
+                   gpu_launches=steps * len(out) + sum(o["teacher_steps"] for o in out))
 
 
-def bench_cycle(args, world, rank, local):
+def bench_cycle(args, world, rank, local, steps):
     """Ragged serving mix: 128 requests with prefix lengths uniform on {0, 32, ..., 8192},
     32-token blocks, 6 hybrid layers (16 query / 4 KV heads, head dim 128, F 256, independent
     W), 8 denoising steps per block then a commit of every layer, captured as one CUDA graph.
@@ -669,20 +753,59 @@ def bench_cycle(args, world, rank, local):
             a = acts[nsteps - 1][l]
             bha.commit_block(cu, a["K"], a["V"], Ws[l], Ss[l], Zs[l], max_block=B, stream=stream)
 
-    ms = max_over_ranks(time_graphed(cycle, args.steps, args.warmup, world, stream), world)
-    if rank == 0:
-        ms_cycle = ms / args.steps
-        nbytes = nsteps * layers * step_bytes() + layers * commit_bytes()
-        cfg = {"workload": "ragged serving mix: 128 requests, prefixes uniform on {0,32,...,8192}, "
-                           "32-token blocks, 6 hybrid layers, 8 denoising steps then a commit per "
-                           "block cycle (one CUDA graph)", "requests": R, "layers": layers,
-               "steps_per_block": nsteps, "prefix_mean": float(plen.mean())}
-        print(json.dumps(_line("serving-cycle tokens/s per denoise step (6 hybrid layers)",
-                               nsteps * R * B * world / (ms_cycle / 1e3), UNIT, args, world,
-                               ms_cycle, True, cfg, dtype="bf16", precision="bf16 activations; fp32 states",
-                               roofline=_roof(nbytes, ms_cycle, peaks, src, "block cycle"),
-                               committed_tokens_per_s=R * B * world / (ms_cycle / 1e3),
-                               gpu_launches=args.steps * (nsteps * layers + layers))), flush=True)
+    ms = max_over_ranks(time_graphed(cycle, steps, args.warmup, world, stream), world)
+    del acts, Ss, Zs
+    torch.cuda.empty_cache()
+    ms_cycle = ms / steps
+    nbytes = nsteps * layers * step_bytes() + layers * commit_bytes()
+    cfg = {"workload": "ragged serving mix: 128 requests, prefixes uniform on {0,32,...,8192}, "
+                       "32-token blocks, 6 hybrid layers, 8 denoising steps then a commit per "
+                       "block cycle (one CUDA graph)", "requests": R, "layers": layers,
+           "steps_per_block": nsteps, "prefix_mean": float(plen.mean())}
+    return _record("serving-cycle tokens/s per denoise step (6 hybrid layers)",
+                   whole_job_rate(nsteps * R * B, steps, ms, world), UNIT, steps, ms_cycle, cfg,
+                   dtype="bf16", precision="bf16 activations; fp32 states",
+                   roofline=_roof(nbytes, ms_cycle, peaks, src, "block cycle"),
+                   committed_tokens_per_s=whole_job_rate(R * B, steps, ms, world),
+                   gpu_launches=steps * (nsteps * layers + layers))
+
+
+def bench_per_qhead(args, world, rank, local, steps):
+    """The decode step in the per-query-head layout (a W and a state per query head: 16 query
+    and 16 state heads), 128 requests, 32-token blocks, fp32 states of 1024-token prefixes
+    built through the library: four times the state bytes of the grouped layout."""
+    from linear_attention_diffusion_hedgehog_b200 import bha
+
+    peaks, src = load_peaks()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(23 + rank)
+    W, cu, sets = make_decode_sets(gen, nsets=NSETS, Hkv=HQ)
+    stream = torch.cuda.Stream()
+    dims = bha.make_dims(R, HQ, HQ, D, F, B, R * B, R, torch.bfloat16)
+    variant = bha.kernel_variant(dims, 1)
+
+    def step(i):
+        s = sets[i % NSETS]
+        bha.hybrid_attn(cu, s["Q"], s["K"], s["V"], s["S"], s["Z"], W, max_block=B, out=s["O"],
+                        stream=stream)
+
+    ms = max_over_ranks(time_graphed(step, steps, args.warmup, world, stream), world)
+    del sets
+    torch.cuda.empty_cache()
+    ms_step = ms / steps
+    cfg = dict(decode_config(), workload="decode step, per-query-head layout: 128 requests x 32-token "
+               "blocks, 16 query heads each with its own W and fp32 state (16 state heads), head dim "
+               "128, feature dim 256, states of 1024-token prefixes", kv_heads=HQ,
+               l2=f"rotating {NSETS} input/state sets of ~340 MB each")
+    return _record("hybrid-attn tokens/s per denoise step, per-query-head states", whole_job_rate(R * B, steps, ms, world),
+                   UNIT, steps, ms_step, cfg, dtype="bf16", kernel_variant=variant,
+                   roofline=_roof(step_bytes(Hkv=HQ), ms_step, peaks, src,
+                                  "hybrid tensor-core" if variant == 1 else "hybrid generic",
+                                  flops=step_flops(Hkv=HQ)),
+                   gpu_launches=steps)
+
+
+SUB_STEPS = {"commit": 1000, "featuremap": 1000, "per_qhead": 1000, "sweep": 500, "cycle": 50}
 
 
 def main():
@@ -691,8 +814,9 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["decode", "commit", "featuremap", "sweep", "cycle"],
-                    default="decode")
+    ap.add_argument("--workload", choices=["all", "decode", "commit", "featuremap", "per_qhead", "sweep",
+                                           "cycle"],
+                    default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
@@ -701,12 +825,26 @@ def main():
         bench_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
         return
     world, rank, local = dist_setup(args.gpus)
+    subs = {"commit": bench_commit, "featuremap": bench_featuremap, "per_qhead": bench_per_qhead,
+            "sweep": bench_sweep, "cycle": bench_cycle}
     try:
-        if args.workload == "decode":
-            bench_decode(args, world, rank, local)
-        else:
-            {"commit": bench_commit, "featuremap": bench_featuremap, "sweep": bench_sweep,
-             "cycle": bench_cycle}[args.workload](args, world, rank, local)
+        if args.workload in subs:
+            rec = subs[args.workload](args, world, rank, local, args.steps)
+            if rank == 0:
+                rec.update({"n_gpus": world, "warmup": args.warmup, "scaling": "weak",
+                            "vs_baseline": None, "data": "synthetic"})
+                print(json.dumps(rec), flush=True)
+            return
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(1234 + rank)
+        line = bench_decode(args, world, rank, local, gen)
+        if args.workload == "all":
+            for name, fn in subs.items():
+                rec = fn(args, world, rank, local, min(args.steps, SUB_STEPS[name]))
+                if rank == 0:
+                    line["workloads"][name] = rec
+        if rank == 0:
+            print(json.dumps(line), flush=True)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -24,6 +24,8 @@
  * - States: S [num_slots][Hkv][F][d] fp32 and Z [num_slots][Hkv][F] fp32, row-major.
  *   Request r uses slot state_slot[r] (DEVICE int32 [R]) or slot r when state_slot is NULL.
  * - W [Hkv][d][F/2] row-major in the activation dtype; alpha [Hq] fp32 or NULL (w = 1).
+ * - Every call works on the CURRENT CUDA device (cudaGetDevice): its launches, tensor maps and
+ *   device limits are those of that device, so all pointers and the stream must belong to it.
  * - All tensor pointers are DEVICE pointers, 16-byte aligned; the caller allocates and owns
  *   every buffer.  The library allocates nothing, keeps no per-call state, never
  *   synchronises the stream, and enqueues its kernels on `stream` (a cudaStream_t; NULL is

@@ -92,8 +92,9 @@ def selftest_bounded_wait(limit_cycles, dev_err, stream=None):
     """Runs the library's bounded wait on an mbarrier that never completes; dev_err (a device
     int32 tensor, zeroed by the caller) receives BHA_ERR_TIMEOUT once the wait gives up."""
     _cuda(dev_err, "dev_err", dtype=torch.int32)
-    st = lib().bha_selftest_bounded_wait(int(limit_cycles), _ptr(dev_err),
-                                         _stream(dev_err.device, stream))
+    with torch.cuda.device(dev_err.device):  # the library uses the current device
+        st = lib().bha_selftest_bounded_wait(int(limit_cycles), _ptr(dev_err),
+                                             _stream(dev_err.device, stream))
     _check(st, "bha_selftest_bounded_wait")
 
 
@@ -156,8 +157,9 @@ def featuremap(x, W, out_dtype=torch.float32, out=None, stream=None):
     _cuda(out, "out", dtype=out_dtype, ndim=3)
     _need(tuple(out.shape) == (T, H, 2 * Fh), "out must be [T, H, F]")
     dims = make_dims(0, Hkv, Hkv, d, 2 * Fh, 1, T, 0, x.dtype)  # R, Hq, slots unused here
-    st = lib().bha_featuremap(ctypes.byref(dims), _ptr(x), H, _ptr(W), _ptr(out),
-                              _DTYPE_CODE[out_dtype], _stream(x.device, stream))
+    with torch.cuda.device(x.device):  # the library uses the current device
+        st = lib().bha_featuremap(ctypes.byref(dims), _ptr(x), H, _ptr(W), _ptr(out),
+                                  _DTYPE_CODE[out_dtype], _stream(x.device, stream))
     _check(st, "bha_featuremap")
     return out
 
@@ -193,9 +195,10 @@ def hybrid_attn(cu_blk, Q, K, V, S, Z, W, *, max_block, alpha=None, state_slot=N
     if dev_err is not None:
         _cuda(dev_err, "dev_err", dtype=torch.int32)
     dims = make_dims(R, Hq, Hkv, d, F, max_block, T, S.shape[0], dt)
-    st = lib().bha_hybrid_attn(ctypes.byref(dims), _ptr(cu_blk), _ptr(state_slot), _ptr(Q),
-                               _ptr(K), _ptr(V), _ptr(S), _ptr(Z), _ptr(W), _ptr(alpha),
-                               _ptr(out), _ptr(dev_err), _stream(Q.device, stream))
+    with torch.cuda.device(Q.device):  # the library uses the current device
+        st = lib().bha_hybrid_attn(ctypes.byref(dims), _ptr(cu_blk), _ptr(state_slot), _ptr(Q),
+                                   _ptr(K), _ptr(V), _ptr(S), _ptr(Z), _ptr(W), _ptr(alpha),
+                                   _ptr(out), _ptr(dev_err), _stream(Q.device, stream))
     _check(st, "bha_hybrid_attn")
     return out
 
@@ -222,9 +225,10 @@ def commit_block(cu_blk, K, V, W, S, Z, *, max_block, state_slot=None, dev_err=N
     if dev_err is not None:
         _cuda(dev_err, "dev_err", dtype=torch.int32)
     dims = make_dims(R, Hkv, Hkv, d, F, max_block, T, S.shape[0], dt)
-    st = lib().bha_commit_block(ctypes.byref(dims), _ptr(cu_blk), _ptr(state_slot), _ptr(K),
-                                _ptr(V), _ptr(W), _ptr(S), _ptr(Z), _ptr(dev_err),
-                                _stream(K.device, stream))
+    with torch.cuda.device(K.device):  # the library uses the current device
+        st = lib().bha_commit_block(ctypes.byref(dims), _ptr(cu_blk), _ptr(state_slot), _ptr(K),
+                                    _ptr(V), _ptr(W), _ptr(S), _ptr(Z), _ptr(dev_err),
+                                    _stream(K.device, stream))
     _check(st, "bha_commit_block")
     return S, Z
 
@@ -257,9 +261,10 @@ def full_prefix_attn(cu_blk, kv_len, Q, Kc, Vc, *, max_block, workspace=None, ou
         _cuda(dev_err, "dev_err", dtype=torch.int32)
     dims = make_dims(R, Hq, Hkv, d, 2, max_block, T, 0, dt)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().bha_full_prefix_attn(ctypes.byref(dims), _ptr(cu_blk), _ptr(kv_len), _ptr(Q),
-                                    _ptr(Kc), _ptr(Vc), cap, _ptr(out), _ptr(workspace), wbytes,
-                                    _ptr(dev_err), _stream(Q.device, stream))
+    with torch.cuda.device(Q.device):  # the library uses the current device
+        st = lib().bha_full_prefix_attn(ctypes.byref(dims), _ptr(cu_blk), _ptr(kv_len), _ptr(Q),
+                                        _ptr(Kc), _ptr(Vc), cap, _ptr(out), _ptr(workspace), wbytes,
+                                        _ptr(dev_err), _stream(Q.device, stream))
     _check(st, "bha_full_prefix_attn")
     return out
 
@@ -287,8 +292,9 @@ def full_prefix_attn_noalloc(cu_blk, kv_len, Q, Kc, Vc, *, max_block, out=None, 
     if dev_err is not None:
         _cuda(dev_err, "dev_err", dtype=torch.int32)
     dims = make_dims(R, Hq, Hkv, d, 2, max_block, T, 0, dt)
-    st = lib().bha_full_prefix_attn_noalloc(ctypes.byref(dims), _ptr(cu_blk), _ptr(kv_len),
-                                            _ptr(Q), _ptr(Kc), _ptr(Vc), cap, _ptr(out),
-                                            _ptr(dev_err), _stream(Q.device, stream))
+    with torch.cuda.device(Q.device):  # the library uses the current device
+        st = lib().bha_full_prefix_attn_noalloc(ctypes.byref(dims), _ptr(cu_blk), _ptr(kv_len),
+                                                _ptr(Q), _ptr(Kc), _ptr(Vc), cap, _ptr(out),
+                                                _ptr(dev_err), _stream(Q.device, stream))
     _check(st, "bha_full_prefix_attn_noalloc")
     return out

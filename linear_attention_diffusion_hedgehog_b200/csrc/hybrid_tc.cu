@@ -1,13 +1,15 @@
 // Tensor-core block-hybrid decode step for sm_100a (bf16 activations, d = 128, F = 256,
-// four query heads per KV head, blocks of up to 32 tokens).
+// G = 1, 2 or 4 query heads per KV head, blocks of up to 32 tokens).
 //
 // Source: "Retrofitting Linear Attention into Diffusion Language Models", §3.1: per query q
 //   sm_num = sum_j exp(q.k_j/sqrt d) v_j,  sm_den = sum_j exp(q.k_j/sqrt d)   (active block)
 //   lin_num = phi(q)^T S,  lin_den = phi(q)^T Z,  phi(q) = [softmax(qW), softmax(-qW)]
 //   out = (w sm_num + lin_num) / (w sm_den + lin_den),  w = sigmoid(alpha_h)
 //
-// Work unit: one (request r, KV head g).  Its 4 query heads x 32 block rows are exactly one
-// 128-row MMA tile (row = 4 t + head-in-group, the order Q has in memory), and they share
+// Work unit: one (request r, KV head g).  Its G query heads x 32 block rows fill 32 G rows of
+// one 128-row MMA tile (row = G t + head-in-group, the order Q has in memory; for G < 4 the
+// other rows hold whatever follows in shared memory and are never stored; with G = 1 this
+// is the per-query-head layout, W and the states per query head), and they share
 // K_g, V_g, W_g, S_g and Z_g, so S_g (128 KiB fp32, the dominant traffic) is read once per
 // unit.  A persistent grid walks the units; unit u is (r = u / Hkv, g = u % Hkv), so a CTA
 // whose grid stride is a multiple of Hkv keeps one W_g resident.
@@ -19,10 +21,12 @@
 // so each group of 32 e values goes to the tensor cores as soon as it exists (fp32 in TMEM,
 // contracted in tf32 against the fp32 S tile exactly as TMA delivered it), and the
 // normalisation by sum e+/-, known only at the end, moves to the epilogue.  A+ and A-
-// accumulate in two TMEM accumulators; P V joins A+ with P pre-scaled by
-// kappa = sum e+ / e^{-m}, which the epilogue's factor e^{-m} / sum e+ undoes:
-//   out = (c+ A+ + c- A-) / den,  c+/- = e^{-m} / sum e+/-,
-//   den = w sum_j P_j + e^{-m} (e+.Z+ / sum e+ + e-.Z- / sum e-).
+// accumulate in two TMEM accumulators; P V joins A+ with P stored as w 2^{s_j} sum e+
+// (s_j the scaled score in log2 units), which the epilogue's factor 1 / sum e+ undoes:
+//   out = (A+ + r A-) / den,  r = sum e+ / sum e-,  den = sum_j P_j + e+.Z+ + r e-.Z-.
+// For large scores both e+ and e- are shifted down by tl = max(0, max_j s_j - 100) (a common
+// factor of the linear branch), so P stays below 2^107; for states that are all zero the
+// linear branch is dropped and P is shifted by max_j s_j instead.
 // TMEM columns: u [0,128), overwritten in place by e+; e- [128,256) (the block scores sit in
 // its top 32 columns until e- overwrites them); A- [256,384); A+ [384,512).
 //
@@ -59,7 +63,7 @@ namespace {
 constexpr int kD = 128;
 constexpr int kF = 256;
 constexpr int kFh = 128;
-constexpr int kG = 4;
+constexpr int kG = 4;            // query heads per KV head that fill the 128-row tile
 constexpr int kBlk = 32;
 constexpr int kM = kG * kBlk;  // 128 tile rows
 constexpr int kChunk = 32;         // F rows of S per chunk = one group of 32 e values
@@ -213,9 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
           g_res = x.g;
         }
         if (k >= 1 && !tc::mbar_wait(&sm.qk_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
-        tc::mbar_arrive_expect_tx(&sm.qk_full, kQBytes + kKBytes);
-        tc::tma_load_3d(sm.q, &p.tm_q, &sm.qk_full, 0, kG * x.g, x.lo);
-        tc::tma_load_3d(sm.q + kQBytes / 2, &p.tm_q, &sm.qk_full, 64, kG * x.g, x.lo);
+        // Q: two d halves of 32 G rows, each at the start of its 16 KiB half of the tile
+        tc::mbar_arrive_expect_tx(&sm.qk_full, (kQBytes / kG) * p.G + kKBytes);
+        tc::tma_load_3d(sm.q, &p.tm_q, &sm.qk_full, 0, p.G * x.g, x.lo);
+        tc::tma_load_3d(sm.q + kQBytes / 2, &p.tm_q, &sm.qk_full, 64, p.G * x.g, x.lo);
         tc::tma_load_3d(sm.k, &p.tm_k, &sm.qk_full, 0, x.g, x.lo);
         tc::tma_load_3d(sm.k + kKBytes / 2, &p.tm_k, &sm.qk_full, 64, x.g, x.lo);
         armed_qk = k & 1;
@@ -358,8 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
     // One warp per TMEM lane quarter, one thread per tile row (its own TMEM lane).  A failed
     // bounded wait ends the loop for the whole warp (the vote keeps its lanes together).
     const int wq = warp & 3;           // TMEM lane quarter this warp may access
-    const int row = wq * 32 + lane;    // tile row = 4 t + head-in-group
-    const int hl = row & 3;
+    const int row = wq * 32 + lane;    // tile row = G t + head-in-group
+    const int hl = row % p.G;
     const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
     const float scale_log2 = 1.4426950408889634f * 0.08838834764831845f;  // log2(e) / sqrt(128)
     const float log2e = 1.4426950408889634f;
@@ -370,9 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.z_full[k & 1], (k >> 1) & 1, abort_flag, lim))) break;
       tc::tc_fence_after();
 
-      // block softmax over the x.n keys of this request (bidirectional, no mask):
-      // a_j = w 2^{s_j log2e / sqrt d - m}; here only the row max m, P itself is formed once
-      // P's scale is known (below, from the scores still in TMEM)
+      // block softmax over the x.n keys of this request (bidirectional, no mask): only the
+      // row max m of s_j = q.k_j log2(e) / sqrt d here; P itself is formed once its scale is
+      // known (below, from the scores still in TMEM)
       float m2;
       {
         float sv[32];
@@ -382,11 +387,24 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           if (j < x.n) mraw = fmaxf(mraw, sv[j]);
-        // m in log2 units, kept in [-6 log2 e, 90] so that 2^{-m} is finite and not tiny
-        m2 = fminf(fmaxf(mraw * scale_log2, -6.f * log2e), 90.f);
+        m2 = mraw * scale_log2;
       }
-      const float wgt = p.alpha ? 1.f / (1.f + expf(-p.alpha[kG * x.g + hl])) : 1.f;
-      const float em = tc::ex2(-m2);
+      const float wgt = p.alpha && row < kBlk * p.G ? 1.f / (1.f + expf(-p.alpha[p.G * x.g + hl])) : 1.f;
+      // Scale of the linear branch (log2 units).  Both branches meet in A+ with P stored as
+      // w 2^{s_j} sum e+, so e+ and e- are shifted down by tl = max(0, m - 100): then every
+      // stored P is below 2^{107} and no e exceeds 1, and when m > 100 the linear branch,
+      // which tl makes smaller still, is in any case below 2^{-90} of the softmax branch.
+      // States that are all zero (no committed block) add nothing: e+ = e- = 0 and P is
+      // shifted by m instead, so a block whose scores are all very negative stays exact.
+      float zmax;
+      {
+        const float* zk0 = sm.z[k & 1];
+        const float4 a = *reinterpret_cast<const float4*>(zk0 + lane * 8);
+        const float4 b = *reinterpret_cast<const float4*>(zk0 + lane * 8 + 4);
+        zmax = warp_max(fmaxf(fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)), fmaxf(fmaxf(b.x, b.y), fmaxf(b.z, b.w))));
+      }
+      const bool lin = zmax > 0.f;
+      const float tl2 = lin ? fmaxf(0.f, m2 - 100.f) : INFINITY;
 
       // max and min of u over the row's 128 features
       float mx = -INFINITY, mn = INFINITY;
@@ -403,12 +421,12 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
         }
       }
 
-      // e+_f = 2^{(u_f - max u) log2e} over u in place, e-_f = 2^{(min u - u_f) log2e}, group by
-      // group, each released to the MMA as soon as the four warps have written it (e- group 3
-      // overwrites the scores, which this thread has read)
-      const float bpl = mx * log2e, bml = mn * log2e;
+      // e+_f = 2^{(u_f - max u) log2e - tl} over u in place, e-_f = 2^{(min u - u_f) log2e - tl},
+      // group by group, each released to the MMA as soon as the four warps have written it
+      // (e- group 3 overwrites the scores, which this thread has read)
+      const float bpl = mx * log2e + tl2, bml = mn * log2e - tl2;
       const float* zk = sm.z[k & 1];
-      float esp = 0.f, esm = 0.f, zsp = 0.f, zsm = 0.f, kappa = 1.f, psum = 0.f;
+      float esp = 0.f, esm = 0.f, zsp = 0.f, zsm = 0.f, psum = 0.f;
       bool vgood = true;
 #pragma unroll 1
       for (int c = 0; c < kGroups; ++c) {
@@ -433,20 +451,21 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
           tc::tmem_st16(tl + kColU + c * 32 + 16 * h, ep);
         }
         if (c == kGroups - 1) {
-          // sum e+ is complete, so P (bf16, scaled by kappa = sum e+ / e^{-m}) is formed now,
-          // from the scores that e- group 3 is about to overwrite.  P's buffer is free once
-          // V has landed (V is reloaded only after the previous P V has completed).
+          // sum e+ is complete, so P (bf16, w 2^{s_j} sum e+, or w 2^{s_j - m} for empty
+          // states) is formed now, from the scores that e- group 3 is about to overwrite.  P's
+          // buffer is free once V has landed (V is reloaded only after the previous P V has
+          // completed).
           vgood = __all_sync(0xffffffffu, tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim));
-          kappa = esp / em;
+          const float lsp = lin ? tc::lg2(esp) : -m2;
           float sv[32];
           tc::tmem_ld32(tl + kColS, sv);
           tc::tmem_wait_ld();
           uint32_t packed[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const float a0 = j < x.n ? wgt * tc::ex2(fmaf(sv[j], scale_log2, -m2)) : 0.f;
-            const float a1 = j + 1 < x.n ? wgt * tc::ex2(fmaf(sv[j + 1], scale_log2, -m2)) : 0.f;
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(a0 * kappa, a1 * kappa);
+            const float a0 = j < x.n ? wgt * tc::ex2(fmaf(sv[j], scale_log2, lsp)) : 0.f;
+            const float a1 = j + 1 < x.n ? wgt * tc::ex2(fmaf(sv[j + 1], scale_log2, lsp)) : 0.f;
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
             psum += __low2float(b2) + __high2float(b2);
             packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
           }
@@ -483,16 +502,18 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
         tc::mbar_arrive(&sm.p_ready);
       }
 
-      // epilogue factors: out = (c+ A+ + c- A-) / den, c+/- = e^{-m} / sum e+/-,
-      // den = w sum_j P_j + e^{-m} (e+.Z+ / sum e+ + e-.Z- / sum e-) with the same rounded P
-      // that the P V product uses; handed to the epilogue warps through a double buffer
+      // epilogue factors: out = f+ A+ + f- A- with, after multiplying numerator and
+      // denominator by sum e+,  den = sum_j P_j + e+.Z+ + (sum e+ / sum e-) e-.Z-,  f+ = 1/den,
+      // f- = (sum e+ / sum e-) / den (every term bounded), using the same rounded P that the
+      // P V product uses; handed to the epilogue warps through a double buffer
       const int fb = k & 1;
       if (k >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(&sm.fin_empty[fb], ((k - 2) >> 1) & 1, abort_flag, lim)))
         break;
-      const float den = psum / kappa + em * (zsp / esp + zsm / esm);
+      const float rpm = lin ? esp / esm : 0.f;
+      const float den = psum + (lin ? zsp + zsm * rpm : 0.f);
       const float inv = den != 0.f ? 1.f / den : 0.f;
-      sm.fin[fb][0][row] = em / esp * inv;
-      sm.fin[fb][1][row] = em / esm * inv;
+      sm.fin[fb][0][row] = inv;
+      sm.fin[fb][1][row] = rpm * inv;
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.fin_full[fb]);
     }
@@ -503,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
     // already work on the next unit.
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
-    const int tok = row >> 2, hl = row & 3;
+    const int tok = row / p.G, hl = row % p.G;  // rows past 32 G have tok >= 32: never stored
     const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
     int ucur = blockIdx.x;
     Unit x{};
@@ -515,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
       const float fp = sm.fin[fb][0][row], fm = sm.fin[fb][1][row];
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.fin_empty[fb]);
-      __nv_bfloat16* orow = p.O + ((size_t)(x.lo + tok) * p.Hq + kG * x.g + hl) * kD;
+      __nv_bfloat16* orow = p.O + ((size_t)(x.lo + tok) * p.Hq + p.G * x.g + hl) * kD;
       const bool live = tok < x.n;
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
@@ -555,7 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
 
 // ----------------------------------------------------------------- host side
 bool hybrid_tc_supports(const HybridArgs& a, bool act_bf16) {
-  return act_bf16 && a.d == kD && a.F == kF && a.Hq == kG * a.Hkv && a.Bmax <= kBlk &&
+  const int G = a.Hkv > 0 && a.Hq % a.Hkv == 0 ? a.Hq / a.Hkv : 0;
+  return act_bf16 && a.d == kD && a.F == kF && (G == 1 || G == 2 || G == kG) && a.Bmax <= kBlk &&
          (long long)a.num_slots * a.Hkv * kF < (1ll << 31);
 }
 
@@ -565,7 +587,7 @@ cudaError_t launch_hybrid_tc(const HybridArgs& a, cudaStream_t st) {
   {
     const uint64_t dims[3] = {kD, (uint64_t)a.Hq, T};
     const uint64_t strides[2] = {kD * 2, (uint64_t)a.Hq * kD * 2};
-    const uint32_t box[3] = {64, kG, kBlk};
+    const uint32_t box[3] = {64, (uint32_t)(a.Hq / a.Hkv), kBlk};
     if (!make_tensor_map(&p.tm_q, false, 3, a.Q, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
   }
   {
@@ -597,6 +619,7 @@ cudaError_t launch_hybrid_tc(const HybridArgs& a, cudaStream_t st) {
   p.R = a.R;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;
+  p.G = a.Hq / a.Hkv;
   p.T = a.T;
   p.Bmax = a.Bmax;
   p.num_slots = a.num_slots;

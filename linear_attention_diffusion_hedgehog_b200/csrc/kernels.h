@@ -59,7 +59,7 @@ struct TcHybridParams {
   const float* alpha;
   __nv_bfloat16* O;
   int32_t* dev_err;
-  int r0, R, Hq, Hkv, T, Bmax, num_slots;  // requests r0 .. r0 + R - 1 of the call
+  int R, Hq, Hkv, G, T, Bmax, num_slots;  // G = Hq / Hkv query heads per KV head
   long long wait_limit;  // SM cycles a bounded wait may spin before giving up
 };
 

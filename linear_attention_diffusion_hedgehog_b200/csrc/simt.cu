@@ -180,15 +180,23 @@ __global__ void __launch_bounds__(128) hybrid_simt(HybridArgs a) {
         if (k < d) num_lin[c] = fmaf(p, srow[k], num_lin[c]);
       }
     }
-    // shared normaliser; the softmax branch carries e^{-m}, so the linear branch does too
-    const float em = expf(-m);
-    const float den = w * den_sm + em * den_lin;
+    // shared normaliser.  The softmax sums carry e^{-m}; both branches are brought to the
+    // common scale e^{-M}, M = max(m, log den_lin), so that neither factor overflows (a
+    // branch that underflows is negligible beside the other); states that are all zero add
+    // nothing (den_lin = 0: the softmax branch alone, unscaled)
+    float fsm = 1.f, flin = 0.f;
+    if (den_lin > 0.f) {
+      const float M = fmaxf(m, logf(den_lin));
+      fsm = expf(m - M);
+      flin = expf(-M);
+    }
+    const float den = w * den_sm * fsm + den_lin * flin;
     T* orow = static_cast<T*>(a.O) + ((size_t)t * a.Hq + h) * d;
 #pragma unroll
     for (int c = 0; c < kDCols; ++c) {
       const int k = lane + 32 * c;
       if (k < d) {
-        const float num = w * num_sm[c] + em * num_lin[c];
+        const float num = w * num_sm[c] * fsm + num_lin[c] * flin;
         orow[k] = from_f32<T>(den != 0.f ? num / den : 0.f);
       }
     }

@@ -485,3 +485,103 @@ def test_bounded_wait_gives_up_and_reports_timeout():
     phi = bha.featuremap(dev(x, torch.bfloat16), dev(W, torch.bfloat16))
     torch.cuda.synchronize()
     _check_phi(host64(phi), ref.featuremap(x, W), torch.float32)
+
+
+# ------------------------------------------------------------------- extreme block logits
+
+def _extreme_logit_case(sign, aligned_all, prefix, seed, dtype="bf16", d=128, F=256, Hq=16, Hkv=4):
+    """Block scores near sign * 100 (natural units).  aligned_all: every key of a request is
+    close to one direction v0 and every query is sign * v0, so all of a row's scores are about
+    sign * 100; otherwise each query copies one key of its block (scaled by sign), so one score
+    per row is about sign * 100 and the rest are O(25).  prefix: states drawn from 700-token
+    prefixes, or all zero."""
+    lens = [32, 17, 1, 32]
+    c = inputs.decode_case(R=4, Hq=Hq, Hkv=Hkv, d=d, F=F, block_lens=lens, prefix_lens=0,
+                           seed=seed, dtype=dtype)
+    rng = np.random.default_rng(seed + 100)
+    rnd = inputs.bf16_round if dtype == "bf16" else (lambda a: a.astype(np.float32))
+    G = Hq // Hkv
+    K = np.empty_like(c.K)
+    Q = np.empty_like(c.Q)
+    amp = np.sqrt(100.0 * np.sqrt(d) / d)  # |q| |k| / sqrt d ~ 100 for unit-variance directions
+    for r in range(4):
+        lo, hi = c.cu_blk[r], c.cu_blk[r + 1]
+        for g in range(Hkv):
+            if aligned_all:
+                v0 = rng.standard_normal(d)
+                K[lo:hi, g] = amp * (v0 + 0.05 * rng.standard_normal((hi - lo, d)))
+                for h in range(G):
+                    Q[lo:hi, g * G + h] = sign * amp * v0
+            else:
+                K[lo:hi, g] = amp * rng.standard_normal((hi - lo, d))
+                for h in range(G):
+                    Q[lo:hi, g * G + h] = sign * K[lo + rng.permutation(hi - lo), g]
+    c.K, c.Q = rnd(K), rnd(Q)
+    if prefix:
+        S_np, Z_np = inputs.random_states(4, Hkv, F, d, prefix_len=700, seed=seed)
+    else:
+        S_np, Z_np = np.zeros((4, Hkv, F, d), np.float32), np.zeros((4, Hkv, F), np.float32)
+    return c, S_np, Z_np
+
+
+@pytest.mark.parametrize("sign,aligned_all,prefix", [
+    (+1, False, False), (+1, False, True), (+1, True, False), (+1, True, True),
+    (-1, True, False), (-1, True, True)])
+def test_decode_step_extreme_block_logits(sign, aligned_all, prefix):
+    """Scores of about +100 overflow exp in fp32 unless shifted, and a row whose scores are
+    all about -100 underflows it: with an empty prefix the output must still be the block
+    softmax, with a prefix the linear branch must dominate (softmax weight ~e^-100); checked
+    against the float64 oracle on the tensor-core path."""
+    c, S_np, Z_np = _extreme_logit_case(sign, aligned_all, prefix, seed=50 + 7 * aligned_all + 3 * prefix)
+    d = bha.make_dims(4, 16, 4, 128, 256, 32, int(c.cu_blk[-1]), 4, torch.bfloat16)
+    assert bha.kernel_variant(d, 1) == 1
+    s = np.einsum("thd,tgd->th", c.Q.reshape(-1, 4, 4, 128).astype(np.float64)[:, :, 0, :],
+                  c.K.astype(np.float64)) / np.sqrt(128.0)
+    assert np.abs(s).max() > 80  # the case really reaches the edge
+    O = run_hybrid(c, dev(S_np, torch.float32), dev(Z_np, torch.float32))
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, S_np.astype(np.float64), Z_np.astype(np.float64), c.W)
+    assert_close(host64(O), want, TOL_BF16, "O")
+
+
+@pytest.mark.parametrize("sign,prefix", [(+1, False), (+1, True), (-1, False), (-1, True)])
+def test_generic_kernel_extreme_block_logits(sign, prefix):
+    """The same edges on the CUDA-core kernel (fp32 activations, all of a row's scores about
+    sign * 100)."""
+    c, S_np, Z_np = _extreme_logit_case(sign, True, prefix, seed=70 + 3 * prefix, dtype="f32",
+                                        d=64, F=64, Hq=4, Hkv=2)
+    O = run_hybrid(c, dev(S_np, torch.float32), dev(Z_np, torch.float32))
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, S_np.astype(np.float64), Z_np.astype(np.float64), c.W)
+    assert_close(host64(O), want, dict(rel_l2=1e-4, rel_max=1e-4), "O")
+
+
+# ------------------------------------------------------------------- query heads per KV head
+
+@pytest.mark.parametrize("Hq,Hkv", [(16, 16), (8, 4)])
+def test_decode_step_one_and_two_query_heads_per_state(Hq, Hkv):
+    """G = Hq / Hkv = 1 is the per-query-head layout (a W and a state per query head), G = 2 a
+    smaller group; both take the tensor-core kernel, whose 128-row tile then holds 32 G live
+    rows.  Ragged blocks, states committed from 64-token prefixes, the gate; every row checked."""
+    lens = [32, 9, 1, 32, 20, 32]
+    c = inputs.decode_case(R=6, Hq=Hq, Hkv=Hkv, d=128, F=256, block_lens=lens, prefix_lens=64,
+                           seed=80 + Hq, dtype="bf16", with_alpha=True)
+    d = bha.make_dims(6, Hq, Hkv, 128, 256, 32, int(c.cu_blk[-1]), 6, torch.bfloat16)
+    assert bha.kernel_variant(d, 1) == 1
+    S, Z = build_states_on_gpu(c, block=32)
+    So, Zo = oracle_states(c)
+    O = run_hybrid(c, S, Z, alpha=c.alpha)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, So, Zo, c.W, c.alpha)
+    assert_close(host64(O), want, TOL_BF16, "O")
+
+
+def test_decode_step_per_query_head_serving_size_sampled():
+    """128 requests with a W and a state per query head (16 / 16 heads), 32-token blocks,
+    states from 256-token prefixes committed through the library; 4 sampled requests."""
+    c = inputs.decode_case(R=128, Hq=16, Hkv=16, d=128, F=256, block_lens=32, prefix_lens=256,
+                           seed=91, dtype="bf16")
+    S, Z = build_states_on_gpu(c, block=32)
+    O = host64(run_hybrid(c, S, Z))
+    reqs = np.random.default_rng(4).choice(128, 4, replace=False)
+    So, Zo = oracle_states(c, reqs)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, So, Zo, c.W)
+    rows = rows_of(c, reqs)
+    assert_close(O[rows], want[rows], TOL_BF16, "O")
