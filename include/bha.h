@@ -96,6 +96,19 @@ int bha_hybrid_attn(const bha_dims* dims, const int32_t* cu_blk, const int32_t* 
                     const float* Z, const void* W, const float* alpha, void* O,
                     int32_t* dev_err, void* stream);
 
+/* The last denoising step of a block fused with that block's commit (§3.1 block commit; §3.3
+ * serves the step "including the causal state update" in one kernel launch).
+ *   Arguments, layouts and dev_err as in bha_hybrid_attn, except that S and Z are updated:
+ *   O is the step's output over the states as passed in (the blocks committed before this
+ *   one), and then, for each request, S += sum_t phi(k_t) v_t^T and Z += sum_t phi(k_t) over
+ *   its block rows, as bha_commit_block does.  Two requests must not name the same slot.
+ * The tensor-core kernel (the dims bha_hybrid_attn takes on tensor cores) reads each state
+ * once for both parts; other dims run the generic decode step and commit as two launches. */
+int bha_hybrid_attn_commit(const bha_dims* dims, const int32_t* cu_blk, const int32_t* state_slot,
+                           const void* Q, const void* K, const void* V, float* S, float* Z,
+                           const void* W, const float* alpha, void* O, int32_t* dev_err,
+                           void* stream);
+
 /* Block commit (§3.1: S_n = S_{n-1} + sum_{t in B_n} phi(k_t) v_t^T, Z_n likewise), in place.
  *   K/V [T][Hkv][d] activation dtype, W [Hkv][d][F/2]; S, Z updated in place (fp32).
  * Any b_r >= 0 is allowed (b_r = 0 leaves the slot untouched).  Two requests must not
@@ -159,7 +172,8 @@ const char* bha_status_string(int status);
 
 /* Which kernel variant a call with these dims takes: 0 = generic CUDA-core kernel,
  * 1 = tensor-core (tcgen05/TMA) kernel.  which: 0 featuremap (for x_heads = num_q_heads),
- * 1 hybrid, 2 commit, 3 full prefix.  Negative on invalid dims. */
+ * 1 hybrid, 2 commit, 3 full prefix, 4 hybrid fused with the commit.  Negative on invalid
+ * dims. */
 int bha_kernel_variant(const bha_dims* dims, int32_t which);
 
 /* Library ABI version (major * 100 + minor). */

@@ -50,6 +50,8 @@ _SIGS = {
                                        _P, _P, _P]),
     "bha_commit_block": (ctypes.c_int, [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P,
                                         _P]),
+    "bha_hybrid_attn_commit": (ctypes.c_int, [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P,
+                                              _P, _P, _P, _P, _P]),
     "bha_full_prefix_attn": (ctypes.c_int, [ctypes.POINTER(Dims), _P, _P, _P, _P, _P,
                                             ctypes.c_int64, _P, _P, ctypes.c_size_t, _P, _P]),
     "bha_full_prefix_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(Dims), ctypes.c_int64]),
@@ -200,6 +202,47 @@ def hybrid_attn(cu_blk, Q, K, V, S, Z, W, *, max_block, alpha=None, state_slot=N
                                    _ptr(K), _ptr(V), _ptr(S), _ptr(Z), _ptr(W), _ptr(alpha),
                                    _ptr(out), _ptr(dev_err), _stream(Q.device, stream))
     _check(st, "bha_hybrid_attn")
+    return out
+
+
+def hybrid_attn_commit(cu_blk, Q, K, V, S, Z, W, *, max_block, alpha=None, state_slot=None,
+                       out=None, dev_err=None, stream=None):
+    """The last denoising step of a block fused with its commit: returns the step's output over
+    the states as passed in, and folds each request's block into S and Z in place."""
+    _cuda(Q, "Q", ndim=3)
+    dt = Q.dtype
+    _cuda(K, "K", dtype=dt, ndim=3)
+    _cuda(V, "V", dtype=dt, ndim=3)
+    _cuda(W, "W", dtype=dt, ndim=3)
+    _cuda(S, "S", dtype=torch.float32, ndim=4)
+    _cuda(Z, "Z", dtype=torch.float32, ndim=3)
+    _cuda(cu_blk, "cu_blk", dtype=torch.int32, ndim=1)
+    T, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    F = S.shape[2]
+    R = cu_blk.shape[0] - 1
+    _need(tuple(K.shape) == (T, Hkv, d) and tuple(V.shape) == (T, Hkv, d), "K/V must be [T, Hkv, d]")
+    _need(tuple(W.shape) == (Hkv, d, F // 2), "W must be [Hkv, d, F/2]")
+    _need(tuple(S.shape[1:]) == (Hkv, F, d) and tuple(Z.shape) == (S.shape[0], Hkv, F),
+          "S must be [slots, Hkv, F, d], Z [slots, Hkv, F]")
+    if alpha is not None:
+        _cuda(alpha, "alpha", dtype=torch.float32, ndim=1)
+        _need(alpha.shape[0] == Hq, "alpha must be [Hq]")
+    if state_slot is not None:
+        _cuda(state_slot, "state_slot", dtype=torch.int32, ndim=1)
+        _need(state_slot.shape[0] == R, "state_slot must be [R]")
+    if out is None:
+        out = torch.empty_like(Q)
+    _cuda(out, "out", dtype=dt, ndim=3)
+    if dev_err is not None:
+        _cuda(dev_err, "dev_err", dtype=torch.int32)
+    dims = make_dims(R, Hq, Hkv, d, F, max_block, T, S.shape[0], dt)
+    with torch.cuda.device(Q.device):  # the library uses the current device
+        st = lib().bha_hybrid_attn_commit(ctypes.byref(dims), _ptr(cu_blk), _ptr(state_slot),
+                                          _ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(Z), _ptr(W),
+                                          _ptr(alpha), _ptr(out), _ptr(dev_err),
+                                          _stream(Q.device, stream))
+    _check(st, "bha_hybrid_attn_commit")
     return out
 
 

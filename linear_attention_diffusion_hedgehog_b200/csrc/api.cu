@@ -67,12 +67,12 @@ const char* bha_status_string(int status) {
 int bha_kernel_variant(const bha_dims* dims, int32_t which) {
   const int s = check_dims(dims);
   if (s != BHA_OK) return s;
-  if (which < 0 || which > 3) return BHA_ERR_INVALID;
+  if (which < 0 || which > 4) return BHA_ERR_INVALID;
   const bool bf16 = dims->act_dtype == BHA_BF16;
   if (which == 0)
     return bha::featuremap_tc_supports(dims->total_tokens, dims->num_q_heads, dims->num_kv_heads,
                                        dims->head_dim, dims->feature_dim, bf16) ? 1 : 0;
-  if (which == 1) {
+  if (which == 1 || which == 4) {
     bha::HybridArgs a{};
     a.R = dims->num_requests;
     a.Hq = dims->num_q_heads;
@@ -143,6 +143,42 @@ int bha_hybrid_attn(const bha_dims* dims, const int32_t* cu_blk, const int32_t* 
   if (bha::hybrid_tc_supports(a, bf16))
     return launch_status(bha::launch_hybrid_tc(a, static_cast<cudaStream_t>(stream)));
   return launch_status(bha::launch_hybrid_simt(a, bf16, static_cast<cudaStream_t>(stream)));
+}
+
+int bha_hybrid_attn_commit(const bha_dims* dims, const int32_t* cu_blk, const int32_t* state_slot,
+                           const void* Q, const void* K, const void* V, float* S, float* Z,
+                           const void* W, const float* alpha, void* O, int32_t* dev_err,
+                           void* stream) {
+  int s = check_dims(dims);
+  if (s != BHA_OK) return s;
+  if (dims->num_requests == 0 || dims->total_tokens == 0) return BHA_OK;
+  if (!index_ok(cu_blk)) return BHA_ERR_INVALID;
+  if (state_slot != nullptr && !aligned(state_slot, 4)) return BHA_ERR_INVALID;
+  if (state_slot == nullptr && dims->num_slots < dims->num_requests) return BHA_ERR_INVALID;
+  if (!tensor_ok(Q) || !tensor_ok(K) || !tensor_ok(V) || !tensor_ok(S) || !tensor_ok(Z) ||
+      !tensor_ok(W) || !tensor_ok(O))
+    return BHA_ERR_INVALID;
+  if (alpha != nullptr && !aligned(alpha, 4)) return BHA_ERR_INVALID;
+  if (dev_err != nullptr && !aligned(dev_err, 4)) return BHA_ERR_INVALID;
+  const void* outs[3] = {O, S, Z};
+  const void* ins[6] = {Q, K, V, W, alpha, cu_blk};
+  for (const void* o : outs)
+    for (const void* i : ins)
+      if (o == i) return BHA_ERR_INVALID;
+  if (O == (void*)S || O == (void*)Z || (void*)S == (void*)Z) return BHA_ERR_INVALID;
+  bha::HybridArgs a{cu_blk, state_slot, Q, K, V, S, Z, W, alpha, O, dev_err,
+                    dims->num_requests, dims->num_q_heads, dims->num_kv_heads, dims->head_dim,
+                    dims->feature_dim, dims->max_block, dims->total_tokens, dims->num_slots};
+  const bool bf16 = dims->act_dtype == BHA_BF16;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (bha::hybrid_tc_supports(a, bf16)) return launch_status(bha::launch_hybrid_commit_tc(a, S, Z, st));
+  // other dims: the decode step, then the commit, as two launches on the same stream
+  const int r = launch_status(bha::launch_hybrid_simt(a, bf16, st));
+  if (r != BHA_OK) return r;
+  bha::CommitArgs c{cu_blk, state_slot, K, V, W, S, Z, dev_err, dims->num_requests,
+                    dims->num_kv_heads, dims->head_dim, dims->feature_dim, dims->max_block,
+                    dims->total_tokens, dims->num_slots};
+  return launch_status(bha::launch_commit_simt(c, bf16, st));
 }
 
 int bha_commit_block(const bha_dims* dims, const int32_t* cu_blk, const int32_t* state_slot,

@@ -63,6 +63,14 @@ struct TcHybridParams {
   long long wait_limit;  // SM cycles a bounded wait may spin before giving up
 };
 
+// Parameters of the decode step fused with the block commit (hybrid_commit_tc.cu): the decode
+// step's, plus S as the target of the commit's reduce-adds and Z for its atomic adds.
+struct TcHybridCommitParams {
+  TcHybridParams h;
+  CUtensorMap tm_sr;
+  float* Zw;
+};
+
 // Parameters of the tensor-core block-commit kernel (commit_tc.cu).
 struct TcCommitParams {
   CUtensorMap tm_k, tm_v, tm_w, tm_s;  // tm_s: S as [rows of F][d] fp32, the reduce-add target
@@ -105,6 +113,8 @@ int device_sm_count();
 // tensor-core kernels
 bool hybrid_tc_supports(const HybridArgs& a, bool act_bf16);
 cudaError_t launch_hybrid_tc(const HybridArgs& a, cudaStream_t st);
+// the decode step of a, then S += phi(K)^T V and Z += sum phi(K) for its blocks (same shapes)
+cudaError_t launch_hybrid_commit_tc(const HybridArgs& a, float* S, float* Z, cudaStream_t st);
 bool commit_tc_supports(const CommitArgs& a, bool act_bf16);
 cudaError_t launch_commit_tc(const CommitArgs& a, cudaStream_t st);
 bool full_prefix_tc_supports(const FullPrefixArgs& a, bool act_bf16);

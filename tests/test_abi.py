@@ -127,8 +127,30 @@ def test_full_prefix_validation():
 
 def test_kernel_variant_query():
     assert bha.kernel_variant(dims(), 1) in (0, 1)
+    assert bha.kernel_variant(dims(), 4) == bha.kernel_variant(dims(), 1)  # fused: same kernels
     assert bha.kernel_variant(dims(F=3), 1) == bha.BHA_ERR_INVALID
     assert bha.kernel_variant(dims(), 9) == bha.BHA_ERR_INVALID
+
+
+def test_fused_step_and_commit_validation():
+    """The fused call checks what bha_hybrid_attn checks, and that no output (O, S, Z) is also
+    an input or another output."""
+    L = bha.lib()
+
+    def call(dm=None, **kw):
+        a = dict(cu=A16, slot=NULL, Q=A16, K=A16b, V=A16c, S=P(0x40000), Z=P(0x50000),
+                 W=P(0x60000), alpha=NULL, O=P(0x70000), err=NULL)
+        a.update(kw)
+        return L.bha_hybrid_attn_commit(ctypes.byref(dm or dims()), a["cu"], a["slot"], a["Q"],
+                                        a["K"], a["V"], a["S"], a["Z"], a["W"], a["alpha"], a["O"],
+                                        a["err"], NULL)
+    assert call(cu=NULL) == bha.BHA_ERR_INVALID
+    assert call(S=MIS) == bha.BHA_ERR_INVALID
+    assert call(O=A16) == bha.BHA_ERR_INVALID           # O aliases Q
+    assert call(S=A16b) == bha.BHA_ERR_INVALID          # S aliases K
+    assert call(Z=P(0x40000)) == bha.BHA_ERR_INVALID    # Z aliases S
+    assert call(dims(num_slots=2)) == bha.BHA_ERR_INVALID  # identity slots need num_slots >= R
+    assert call(dims(R=0)) == bha.BHA_OK                # nothing to do: no launch
 
 
 def test_selftest_bounded_wait_rejects_bad_arguments_before_launching():

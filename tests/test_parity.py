@@ -585,3 +585,86 @@ def test_decode_step_per_query_head_serving_size_sampled():
     want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, So, Zo, c.W)
     rows = rows_of(c, reqs)
     assert_close(O[rows], want[rows], TOL_BF16, "O")
+
+
+# ------------------------------------------------------------------- decode step fused with the commit
+
+def _run_fused(c, S, Z, alpha=None, state_slot=None, dtype=None):
+    dtype = dtype or act_dtype(c)
+    cu = torch.tensor(c.cu_blk, dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    O = bha.hybrid_attn_commit(cu, dev(c.Q, dtype), dev(c.K, dtype), dev(c.V, dtype), S, Z,
+                               dev(c.W, dtype), max_block=int(max(c.block_lens.max(), 1)),
+                               alpha=None if alpha is None else dev(alpha, torch.float32),
+                               state_slot=state_slot, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0, bha.status_string(int(err.item()))
+    return O
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(16, 4), (16, 16)])
+def test_fused_step_and_commit_ragged_slots_gate(Hq, Hkv):
+    """The last step of a block with its commit in one call: ragged blocks (0, 1, 31, 32
+    tokens), a permuted slot map, the gate and drawn states.  The output reads the states as
+    passed in; afterwards S and Z hold them plus each request's block, as the oracle's commit
+    gives (slots no request names stay as they were)."""
+    lens = [32, 0, 1, 31, 17, 32, 8, 2]
+    c = inputs.decode_case(R=8, Hq=Hq, Hkv=Hkv, d=128, F=256, block_lens=lens, prefix_lens=0,
+                           seed=61 + Hkv, dtype="bf16", with_alpha=True)
+    d = bha.make_dims(8, Hq, Hkv, 128, 256, 32, int(c.cu_blk[-1]), 10, torch.bfloat16)
+    assert bha.kernel_variant(d, 4) == 1
+    S_np, Z_np = inputs.random_states(10, Hkv, 256, 128, prefix_len=700, seed=12)
+    slots = np.array([3, 9, 0, 5, 1, 2, 8, 6], dtype=np.int32)
+    S, Z = dev(S_np, torch.float32), dev(Z_np, torch.float32)
+    O = _run_fused(c, S, Z, alpha=c.alpha, state_slot=torch.tensor(slots, device="cuda"))
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, S_np, Z_np, c.W, c.alpha, slots)
+    assert_close(host64(O), want, TOL_BF16, "O")
+    So, Zo = ref.commit_block(c.cu_blk, c.K, c.V, c.W, S_np, Z_np, slots)
+    assert_close(host64(S), So, TOL_BF16, "S")
+    assert_close(host64(Z), Zo, TOL_BF16, "Z")
+    for untouched in (4, 7, 9):  # slot 9 holds an empty block, slots 4 and 7 no request
+        np.testing.assert_array_equal(host64(S[untouched]), S_np[untouched])
+
+
+def test_fused_step_and_commit_many_units_per_cta_matches_separate_calls():
+    """600 requests (about 17 units per CTA), states committed from 64-token prefixes: the
+    fused call's output equals the decode-only call's bit for bit (same kernel arithmetic),
+    and its states match a separate commit's and, for 6 sampled requests, the oracle's."""
+    c = inputs.decode_case(R=600, Hq=16, Hkv=4, d=128, F=256, block_lens=32, prefix_lens=64,
+                           seed=63, dtype="bf16")
+    S, Z = build_states_on_gpu(c, block=32)
+    S2, Z2 = S.clone(), Z.clone()
+    O_sep = run_hybrid(c, S2, Z2)
+    cu = torch.tensor(c.cu_blk, dtype=torch.int32, device="cuda")
+    bha.commit_block(cu, dev(c.K, torch.bfloat16), dev(c.V, torch.bfloat16),
+                     dev(c.W, torch.bfloat16), S2, Z2, max_block=32)
+    O = _run_fused(c, S, Z)
+    assert torch.equal(O, O_sep)
+    assert_close(host64(S), host64(S2), TOL_BF16, "S vs separate commit")
+    assert_close(host64(Z), host64(Z2), TOL_BF16, "Z vs separate commit")
+    reqs = np.random.default_rng(7).choice(600, 6, replace=False)
+    for r in reqs:
+        lo, hi = c.cu_pre[r], c.cu_pre[r + 1]
+        b0, b1 = c.cu_blk[r], c.cu_blk[r + 1]
+        for g in range(4):
+            Kall = np.concatenate([c.K_pre[lo:hi, g], c.K[b0:b1, g]])
+            Vall = np.concatenate([c.V_pre[lo:hi, g], c.V[b0:b1, g]])
+            So, Zo = ref.state_from_tokens(Kall, Vall, c.W[g])
+            assert_close(host64(S[r, g]), So, TOL_BF16, f"S[{r},{g}]")
+            assert_close(host64(Z[r, g]), Zo, TOL_BF16, f"Z[{r},{g}]")
+
+
+def test_fused_step_and_commit_generic_dims():
+    """Dims outside the tensor-core kernel (fp32, small odd sizes) take the generic decode step
+    and commit as two launches; same results against the oracle."""
+    c = inputs.decode_case(R=3, Hq=6, Hkv=2, d=24, F=20, block_lens=[7, 1, 13], prefix_lens=[9, 0, 30],
+                           seed=65, dtype="f32", with_alpha=True)
+    assert bha.kernel_variant(bha.make_dims(3, 6, 2, 24, 20, 13, 21, 3, torch.float32), 4) == 0
+    S, Z = build_states_on_gpu(c, block=16)
+    So, Zo = oracle_states(c)
+    O = _run_fused(c, S, Z, alpha=c.alpha)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, So, Zo, c.W, c.alpha)
+    assert_close(host64(O), want, TOL_F32, "O")
+    S1, Z1 = ref.commit_block(c.cu_blk, c.K, c.V, c.W, So, Zo)
+    assert_close(host64(S), S1, TOL_F32, "S")
+    assert_close(host64(Z), Z1, TOL_F32, "Z")

@@ -86,8 +86,8 @@ def test_prefix_sweep_states_from_long_prefixes(P, block):
 
 @pytest.mark.parametrize("P", [8192, 32768])
 def test_prefix_sweep_teacher_long_caches(P):
-    """The softmax teacher at 64 requests over caches of P + 32 tokens (split into key ranges
-    and combined); every row of 2 sampled requests against the oracle."""
+    """The softmax teacher at 64 requests over caches of P + 32 tokens (at 32K split into key
+    ranges and combined); every row of 2 sampled requests against the oracle."""
     R, L = 64, P + B
     gen = torch.Generator(device="cuda")
     gen.manual_seed(7 * P)
@@ -96,7 +96,9 @@ def test_prefix_sweep_teacher_long_caches(P):
     Q = torch.randn((R * B, HQ, D), generator=gen, device="cuda").to(BF)
     cu = torch.arange(0, (R + 1) * B, B, dtype=torch.int32, device="cuda")
     kv_len = torch.full((R,), L, dtype=torch.int32, device="cuda")
-    assert bha.full_prefix_workspace_bytes(R, HQ, HKV, D, B, R * B, L) > 0  # split path
+    # 64 requests x 4 KV heads fill the GPU up to 8K-token caches (one key range each); the
+    # 32K cache is split into key ranges whose partials are combined
+    assert (bha.full_prefix_workspace_bytes(R, HQ, HKV, D, B, R * B, L) > 0) == (P == 32768)
     O = host64(bha.full_prefix_attn(cu, kv_len, Q, Kc, Vc, max_block=B))
     for r in np.random.default_rng(P + 1).choice(R, 2, replace=False):
         sl = slice(B * r, B * r + B)
