@@ -2,7 +2,7 @@
 """Throughput of the block-hybrid attention decode step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload all|decode|commit|featuremap|per_qhead|sweep|cycle]
+                    [--workload all|decode|commit|fused|featuremap|per_qhead|sweep|cycle]
 
 Headline workload ("decode"): one denoising step of one block-hybrid layer for 128 requests
 with 32-token active blocks, 16 query / 4 KV heads, head dim 128, feature dim 256 (W is
@@ -20,10 +20,11 @@ against a 126 MB L2).  Multi-GPU runs are independent replicas (no collective on
 
 The default run ("all") adds, under "workloads", one record per other workload, each timed
 the same way with its own roofline: the gated decode step, the block commit (128 requests x
-4 KV heads), the standalone feature map, the per-query-head layout (16 state heads), the prefix sweep (decode step on states committed
+4 KV heads), the last step of a block fused with its commit, the standalone feature map, the per-query-head layout (16 state heads), the prefix sweep (decode step on states committed
 from each prefix vs the in-run softmax teacher over the same cache, 64 requests, prefixes
 512..32768, with the teacher's linear fit) and the serving cycle (ragged mix of 128 requests,
-6 layers, 8 denoising steps then a commit, as one CUDA graph), plus the state-vs-KV-cache
+6 layers, 8 denoising steps then a commit, as one CUDA graph, and again with each layer's
+last step fused with its commit), plus the state-vs-KV-cache
 capacity figures.  --workload X runs one of them alone.
 """
 from __future__ import annotations
@@ -619,6 +620,46 @@ def bench_featuremap(args, world, rank, local, steps):
                    gpu_launches=steps)
 
 
+def fused_bytes(R=R, Hq=HQ, Hkv=HKV, d=D, F=F, B=B):
+    """The last step of a block fused with its commit: the decode step's bytes plus S and Z
+    written back once (the commit's K, V and W are the step's own, already counted)."""
+    return step_bytes(R, Hq, Hkv, d, F, B) + R * Hkv * (F * d * 4 + F * 4)
+
+
+def bench_fused(args, world, rank, local, steps):
+    """The last denoising step of a block fused with its commit (one call), at the decode
+    step's shape: 128 requests, 16 query / 4 KV heads, 32-token blocks; S and Z updated in
+    place, 4 rotating sets."""
+    from linear_attention_diffusion_hedgehog_b200 import bha
+
+    peaks, src = load_peaks()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(29 + rank)
+    W, cu, sets = make_decode_sets(gen)
+    stream = torch.cuda.Stream()
+    dims = bha.make_dims(R, HQ, HKV, D, F, B, R * B, R, torch.bfloat16)
+    variant = bha.kernel_variant(dims, 4)
+
+    def step(i):
+        s = sets[i % NSETS]
+        bha.hybrid_attn_commit(cu, s["Q"], s["K"], s["V"], s["S"], s["Z"], W, max_block=B,
+                               out=s["O"], stream=stream)
+
+    ms = max_over_ranks(time_graphed(step, steps, args.warmup, world, stream), world)
+    del sets
+    torch.cuda.empty_cache()
+    ms_step = ms / steps
+    cfg = dict(decode_config(), workload="last denoising step of a block fused with its commit: 128 "
+               "requests x 32-token blocks, 16 query / 4 KV heads, head dim 128, feature dim 256; "
+               "S and Z updated in place")
+    return _record("block-end step + commit tokens/s (128 reqs)", whole_job_rate(R * B, steps, ms, world),
+                   UNIT, steps, ms_step, cfg, dtype="bf16", kernel_variant=variant,
+                   separate_calls_bytes=step_bytes() + commit_bytes(),
+                   roofline=_roof(fused_bytes(), ms_step, peaks, src,
+                                  "hybrid + commit tensor-core" if variant == 1 else "generic"),
+                   gpu_launches=steps)
+
+
 def linear_fit(xs, ys):
     """Least-squares y = a + b x and its coefficient of determination R^2."""
     xs, ys = np.asarray(xs, np.float64), np.asarray(ys, np.float64)
@@ -753,11 +794,31 @@ def bench_cycle(args, world, rank, local, steps):
             a = acts[nsteps - 1][l]
             bha.commit_block(cu, a["K"], a["V"], Ws[l], Ss[l], Zs[l], max_block=B, stream=stream)
 
+    def cycle_fused(i):
+        # the same cycle with each layer's last step and commit in one call
+        for st in range(nsteps):
+            for l in range(layers):
+                a = acts[st][l]
+                if st < nsteps - 1:
+                    bha.hybrid_attn(cu, a["Q"], a["K"], a["V"], Ss[l], Zs[l], Ws[l], max_block=B,
+                                    out=O, stream=stream)
+                else:
+                    bha.hybrid_attn_commit(cu, a["Q"], a["K"], a["V"], Ss[l], Zs[l], Ws[l],
+                                           max_block=B, out=O, stream=stream)
+
     ms = max_over_ranks(time_graphed(cycle, steps, args.warmup, world, stream), world)
+    ms_fused = max_over_ranks(time_graphed(cycle_fused, steps, args.warmup, world, stream), world)
     del acts, Ss, Zs
     torch.cuda.empty_cache()
     ms_cycle = ms / steps
+    ms_cycle_fused = ms_fused / steps
     nbytes = nsteps * layers * step_bytes() + layers * commit_bytes()
+    nbytes_fused = (nsteps - 1) * layers * step_bytes() + layers * fused_bytes()
+    fused = {"ms_per_cycle": ms_cycle_fused,
+             "tokens_per_s_per_step": whole_job_rate(nsteps * R * B, steps, ms_fused, world),
+             "roofline": _roof(nbytes_fused, ms_cycle_fused, peaks, src,
+                               "block cycle, last step fused with the commit"),
+             "gpu_launches": steps * nsteps * layers}
     cfg = {"workload": "ragged serving mix: 128 requests, prefixes uniform on {0,32,...,8192}, "
                        "32-token blocks, 6 hybrid layers, 8 denoising steps then a commit per "
                        "block cycle (one CUDA graph)", "requests": R, "layers": layers,
@@ -767,6 +828,7 @@ def bench_cycle(args, world, rank, local, steps):
                    dtype="bf16", precision="bf16 activations; fp32 states",
                    roofline=_roof(nbytes, ms_cycle, peaks, src, "block cycle"),
                    committed_tokens_per_s=whole_job_rate(R * B, steps, ms, world),
+                   fused_last_step=fused,
                    gpu_launches=steps * (nsteps * layers + layers))
 
 
@@ -805,7 +867,8 @@ def bench_per_qhead(args, world, rank, local, steps):
                    gpu_launches=steps)
 
 
-SUB_STEPS = {"commit": 1000, "featuremap": 1000, "per_qhead": 1000, "sweep": 500, "cycle": 50}
+SUB_STEPS = {"commit": 1000, "fused": 1000, "featuremap": 1000, "per_qhead": 1000, "sweep": 500,
+             "cycle": 50}
 
 
 def main():
@@ -814,8 +877,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["all", "decode", "commit", "featuremap", "per_qhead", "sweep",
-                                           "cycle"],
+    ap.add_argument("--workload", choices=["all", "decode", "commit", "fused", "featuremap", "per_qhead",
+                                           "sweep", "cycle"],
                     default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -825,8 +888,8 @@ def main():
         bench_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
         return
     world, rank, local = dist_setup(args.gpus)
-    subs = {"commit": bench_commit, "featuremap": bench_featuremap, "per_qhead": bench_per_qhead,
-            "sweep": bench_sweep, "cycle": bench_cycle}
+    subs = {"commit": bench_commit, "fused": bench_fused, "featuremap": bench_featuremap,
+            "per_qhead": bench_per_qhead, "sweep": bench_sweep, "cycle": bench_cycle}
     try:
         if args.workload in subs:
             rec = subs[args.workload](args, world, rank, local, args.steps)

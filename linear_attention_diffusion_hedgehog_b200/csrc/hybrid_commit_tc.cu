@@ -15,15 +15,16 @@
 //                                  ring stage the unit's last state group has released; the
 //                                  other rows are ignored), N 128, into the feature-map
 //                                  columns the unit has finished with
-//   phi  = [softmax(u_k), softmax(-u_k)] per block row by the feature-map warp of lane
-//          quarter 0, rounded to bf16 into that same stage (the producer holds it back until
-//          the commit is done); rows past the block are zero
+//   phi  = [softmax(u_k), softmax(-u_k)] per block row, 8 rows per feature-map warp,
+//          rounded to bf16 into that same stage (the producer holds it back until dS^T and
+//          dZ have read it); rows past the block are zero
 //   dZ   = column sums of the bf16 phi, added to Z with reducing atomics
 //   dS^T = V^T phi                 bf16 MMA, M 128 (d), N 256 (F), K 32, into the accumulator
 //                                  columns once the epilogue has read the output
-//   S   += dS                      the epilogue warps stage dS^T 16 rows of F at a time and
-//                                  add it into S by TMA reduce-add; the lines were read by this
-//                                  unit's state stream moments before, so L2 serves the
+//   S   += dS                      the epilogue warps add dS^T into S with reducing atomics
+//                                  straight from TMEM (lane = d: each warp instruction is one
+//                                  128-byte row piece); the lines were read by this unit's
+//                                  state stream moments before, so L2 serves the
 //                                  read-modify-write and S crosses HBM once each way.
 // The next unit's u and s are issued once phi is in shared memory, so its feature map runs
 // while dS^T is formed and drained.
@@ -71,7 +72,6 @@ constexpr uint32_t kIdPV = tc::instr_desc(1, 0, 1, kM, kD);    // bf16, B MN-maj
 constexpr uint32_t kIdES = tc::instr_desc(2, 0, 1, kM, kD);    // tf32, A from TMEM, B MN-major
 constexpr uint32_t kIdVP = tc::instr_desc(1, 1, 1, kD, kF);    // bf16, A MN-major (V^T), B MN-major
 constexpr uint32_t kPhiBytes = kBlk * kF * 2;  // 16 KiB: [F quarter][32 rows][128 B]
-constexpr int kRedRows = 16;                    // F rows per reduce-add tile
 constexpr int kCommitStage = kStages - 1;       // ring stage lent to the commit
 
 struct __align__(1024) Smem {
@@ -162,10 +162,10 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
     tc::mbar_init(&sm.pv_done, 1);
     tc::mbar_init(&sm.kc_full, 1);
     tc::mbar_init(&sm.uk_done, 1);
-    tc::mbar_init(&sm.phi_ready, 1);    // the feature-map warp of lane quarter 0
+    tc::mbar_init(&sm.phi_ready, 4);    // the four feature-map warps, 8 block rows each
     tc::mbar_init(&sm.ds_full, 1);
     tc::mbar_init(&sm.ds_empty, 4);     // the four epilogue warps
-    tc::mbar_init(&sm.commit_done, 8);  // the epilogue (drain) and feature-map (dZ) warps
+    tc::mbar_init(&sm.commit_done, 4);  // the feature-map warps, done reading phi
     sm.abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
     tc::prefetch_tensormap(&p.tm_v);
     tc::prefetch_tensormap(&p.tm_w);
     tc::prefetch_tensormap(&p.tm_s);
-    tc::prefetch_tensormap(&pc.tm_sr);
+    tc::prefetch_tensormap(&pc.tm_k8);
   }
   if (warp == 1) {
     tc::tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -193,13 +193,17 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
       uint32_t w_loads = 0;
       int armed_qk = -1, armed_v = -1, armed_w = -1, armed_z[2] = {-1, -1}, armed_kc = -1;
       Unit xp{};  // the previous unit: its K is loaded again for its commit
-      // K of unit j into the lent ring stage, laid out like Q (two d halves 16 KiB apart, the
-      // 32 block rows first), once unit j's contraction and P V are done with the stage
+      // K of unit j into the lent ring stage, laid out like Q (two d halves 16 KiB apart), block
+      // rows 8 jq .. 8 jq + 7 at tile rows 32 jq .. (so each TMEM lane quarter of u_k holds 8 of
+      // them), once unit j's contraction and P V are done with the stage
       auto load_kc = [&](const Unit& y, int j) -> bool {
         if (!tc::mbar_wait(&sm.pv_done, j & 1, abort_flag, lim)) return false;
         tc::mbar_arrive_expect_tx(&sm.kc_full, kKBytes);
-        tc::tma_load_3d(sm.s[kCommitStage][0], &p.tm_k, &sm.kc_full, 0, y.g, y.lo);
-        tc::tma_load_3d(sm.s[kCommitStage][1], &p.tm_k, &sm.kc_full, 64, y.g, y.lo);
+#pragma unroll
+        for (int jq = 0; jq < 4; ++jq) {
+          tc::tma_load_3d(sm.s[kCommitStage][0] + jq * 4096, &pc.tm_k8, &sm.kc_full, 0, y.g, y.lo + 8 * jq);
+          tc::tma_load_3d(sm.s[kCommitStage][1] + jq * 4096, &pc.tm_k8, &sm.kc_full, 64, y.g, y.lo + 8 * jq);
+        }
         armed_kc = j & 1;
         return true;
       };
@@ -562,8 +566,10 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.uk_done, k & 1, abort_flag, lim))) break;
       tc::tc_fence_after();
       uint8_t* phib = sm.s[kCommitStage][0];
-      if (wq == 0) {
-        const int t = lane;
+      {
+        // lanes 0-7 of each quarter hold block rows 8 wq + lane; the other lanes skip the math
+        const int t = 8 * wq + (lane & 7);
+        const bool mine = lane < 8;
         float cmx = -INFINITY, cmn = INFINITY;
 #pragma unroll 1
         for (int c = 0; c < kGroups; ++c) {
@@ -583,19 +589,21 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
           float uu[32], e2[32];
           tc::tmem_ld32(tl + kColU + c * 32, uu);
           tc::tmem_wait_ld();
+          if (mine) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float a = uu[i] * log2e;
-            uu[i] = tc::ex2(a - cbx);
-            e2[i] = tc::ex2(cbn - a);
-            csp += uu[i];
-            csm += e2[i];
+            for (int i = 0; i < 32; ++i) {
+              const float a = uu[i] * log2e;
+              uu[i] = tc::ex2(a - cbx);
+              e2[i] = tc::ex2(cbn - a);
+              csp += uu[i];
+              csm += e2[i];
+            }
           }
           tc::tmem_st32(tl + kColU + c * 32, uu);
           tc::tmem_st32(tl + kColEm + c * 32, e2);
         }
         tc::tmem_wait_st();
-        const bool live = t < x.n;  // rows past the block add nothing
+        const bool live = mine && t < x.n;  // rows past the block add nothing
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           const float sc = live ? 1.f / (h ? csm : csp) : 0.f;
@@ -604,22 +612,24 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
             float ee[32];
             tc::tmem_ld32(tl + (h ? kColEm : kColU) + c * 32, ee);
             tc::tmem_wait_ld();
-            uint8_t* rowp = phib + (2 * h + (c >> 1)) * (kPhiBytes / 4) + t * 128;
+            if (mine) {
+              uint8_t* rowp = phib + (2 * h + (c >> 1)) * (kPhiBytes / 4) + t * 128;
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const int ch = 4 * (c & 1) + q4;
-              *reinterpret_cast<uint4*>(rowp + ((ch ^ (t & 7)) << 4)) =
-                  make_uint4(pack_bf16(ee[8 * q4] * sc, ee[8 * q4 + 1] * sc),
-                             pack_bf16(ee[8 * q4 + 2] * sc, ee[8 * q4 + 3] * sc),
-                             pack_bf16(ee[8 * q4 + 4] * sc, ee[8 * q4 + 5] * sc),
-                             pack_bf16(ee[8 * q4 + 6] * sc, ee[8 * q4 + 7] * sc));
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const int ch = 4 * (c & 1) + q4;
+                *reinterpret_cast<uint4*>(rowp + ((ch ^ (t & 7)) << 4)) =
+                    make_uint4(pack_bf16(ee[8 * q4] * sc, ee[8 * q4 + 1] * sc),
+                               pack_bf16(ee[8 * q4 + 2] * sc, ee[8 * q4 + 3] * sc),
+                               pack_bf16(ee[8 * q4 + 4] * sc, ee[8 * q4 + 5] * sc),
+                               pack_bf16(ee[8 * q4 + 6] * sc, ee[8 * q4 + 7] * sc));
+              }
             }
           }
         }
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&sm.phi_ready);  // phi complete (for the MMA and dZ)
+        if (lane == 0) tc::mbar_arrive(&sm.phi_ready);  // this warp's 8 rows of phi are written
       }
       // dZ: column sums of the bf16 phi over the block rows (features tid and tid + 128)
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.phi_ready, k & 1, abort_flag, lim))) break;
@@ -649,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
     const int row = wq * 32 + lane;
     const int tok = row / p.G, hl = row % p.G;  // rows past 32 G have tok >= 32: never stored
     const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
-    int ucur = blockIdx.x, nred = 0;
+    int ucur = blockIdx.x;
     Unit x{};
     for (int k = 0; next_unit(p, units, &ucur, false, &x); ++k) {
       const int fb = k & 1;
@@ -686,43 +696,28 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
         }
       }
 
-      // ---- the commit of this unit: S[f][d] += dS^T[d][f], 16 rows of F at a time staged in
-      // the lent stage ([16 rows][32 d] per tile, two tiles per warp) and added by TMA reduce-add
+      // ---- the commit of this unit: S[f][d] += dS^T[d][f] by reducing atomic adds straight
+      // from the accumulator (lane = d, so each warp instruction adds one 128-byte row piece)
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.ds_full, k & 1, abort_flag, lim))) break;
       tc::tc_fence_after();
       {
-        const int srow0 = (x.slot * p.Hkv + x.g) * kF;
-        uint8_t* stg = sm.s[kCommitStage][1] + wq * 4096;
+        float* Srow = pc.Sw + ((size_t)(x.slot * p.Hkv + x.g) * kF) * kD + wq * 32 + lane;
 #pragma unroll 1
-        for (int j = 0; j < kF / kRedRows; ++j, ++nred) {
-          float dv[kRedRows];
-          tc::tmem_ld16(tl + kColAm + j * kRedRows, dv);
-          // the tile's previous reduce (two tiles back) has read it
-          if (lane == 0 && nred >= 2) tc::bulk_wait_read<1>();
-          __syncwarp();
+        for (int c = 0; c < kF / 32; ++c) {
+          float dv[32];
+          tc::tmem_ld32(tl + kColAm + c * 32, dv);
           tc::tmem_wait_ld();
-          float* tile = reinterpret_cast<float*>(stg + (nred & 1) * (kRedRows * 32 * 4));
-#pragma unroll
-          for (int i = 0; i < kRedRows; ++i) tile[i * 32 + lane] = dv[i];
-          tc::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tc::tma_reduce_add_2d(&pc.tm_sr, tile, wq * 32, srow0 + j * kRedRows);
-            tc::bulk_commit();
+          if (c == kF / 32 - 1) {
+            // dS^T has been read: the next unit's MMAs may overwrite the accumulator columns
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.ds_empty);
           }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) atomicAdd(Srow + (size_t)(c * 32 + i) * kD, dv[i]);
         }
       }
-      // dS^T has been read: the next unit's MMAs may overwrite the accumulator columns
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sm.ds_empty);
-      // the staging tiles have been read: the lent stage may take the next S pair
-      if (lane == 0) tc::bulk_wait_read<0>();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sm.commit_done);
     }
-    // every reduce this warp started has completed (its adds performed)
-    if (lane == 0) tc::bulk_wait_all();
   }
 
   tc::tc_fence_before();
@@ -766,12 +761,13 @@ cudaError_t launch_hybrid_commit_tc(const HybridArgs& a, float* S, float* Z, cud
     if (!make_tensor_map(&p.tm_s, true, 2, a.S, dims, strides, box, kTma128BAtom32)) return cudaErrorInvalidValue;
   }
   {
-    // reduce-add target: S as rows of d fp32 values, 16 x 32 boxes (one warp's tile)
-    const uint64_t dims[2] = {kD, (uint64_t)a.num_slots * a.Hkv * kF};
-    const uint64_t strides[1] = {kD * 4};
-    const uint32_t box[2] = {32, kRedRows};
-    if (!make_tensor_map(&pc.tm_sr, true, 2, S, dims, strides, box, kTmaNone)) return cudaErrorInvalidValue;
+    // K again for the commit, 8 block rows per box
+    const uint64_t dims[3] = {kD, (uint64_t)a.Hkv, T};
+    const uint64_t strides[2] = {kD * 2, (uint64_t)a.Hkv * kD * 2};
+    const uint32_t box[3] = {64, 1, 8};
+    if (!make_tensor_map(&pc.tm_k8, false, 3, a.K, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
   }
+  pc.Sw = S;
   pc.Zw = Z;
   p.cu_blk = a.cu_blk;
   p.state_slot = a.state_slot;

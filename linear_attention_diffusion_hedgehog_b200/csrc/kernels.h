@@ -64,10 +64,11 @@ struct TcHybridParams {
 };
 
 // Parameters of the decode step fused with the block commit (hybrid_commit_tc.cu): the decode
-// step's, plus S as the target of the commit's reduce-adds and Z for its atomic adds.
+// step's, plus K in 8-row boxes for the commit, and S and Z for its atomic adds.
 struct TcHybridCommitParams {
   TcHybridParams h;
-  CUtensorMap tm_sr;
+  CUtensorMap tm_k8;
+  float* Sw;
   float* Zw;
 };
 

@@ -43,3 +43,12 @@ def test_teacher_bytes_over_the_prefix_sweep():
     for P, want in ((512, 88_080_384), (2048, 289_406_976), (8192, 1_094_713_344),
                     (32768, 4_315_938_816)):
         assert b.teacher_bytes(64, 16, 4, 128, 32, P) == 16_777_216 + 131_072 * (P + 32) == want
+
+
+def test_fused_step_and_commit_bytes():
+    """The fused call moves the decode step's bytes plus one write of S and Z; the separate
+    calls move the decode step's bytes plus the commit's (S and Z read and written, K, V, W)."""
+    b = _bench()
+    R, Hkv, d, F = 128, 4, 128, 256
+    assert b.fused_bytes() == b.step_bytes() + R * Hkv * (F * d * 4 + F * 4) == 177_340_416
+    assert b.step_bytes() + b.commit_bytes() - b.fused_bytes() == 76_152_832  # S read + Z + K, V, W
