@@ -656,7 +656,8 @@ def bench_fused(args, world, rank, local, steps):
                    UNIT, steps, ms_step, cfg, dtype="bf16", kernel_variant=variant,
                    separate_calls_bytes=step_bytes() + commit_bytes(),
                    roofline=_roof(fused_bytes(), ms_step, peaks, src,
-                                  "hybrid + commit tensor-core" if variant == 1 else "generic"),
+                                  "hybrid + commit tensor-core" if variant == 1 else "generic",
+                                  traffic=_traffic_for("fused", variant, "hybrid_commit_tc.cu")),
                    gpu_launches=steps)
 
 

@@ -96,8 +96,8 @@ int bha_hybrid_attn(const bha_dims* dims, const int32_t* cu_blk, const int32_t* 
                     const float* Z, const void* W, const float* alpha, void* O,
                     int32_t* dev_err, void* stream);
 
-/* The last denoising step of a block fused with that block's commit (§3.1 block commit; §3.3
- * serves the step "including the causal state update" in one kernel launch).
+/* The last denoising step of a block fused with that block's commit (§3.1 block commit; in
+ * §3.3 one kernel launch per step also performs the state update).
  *   Arguments, layouts and dev_err as in bha_hybrid_attn, except that S and Z are updated:
  *   O is the step's output over the states as passed in (the blocks committed before this
  *   one), and then, for each request, S += sum_t phi(k_t) v_t^T and Z += sum_t phi(k_t) over

@@ -6,7 +6,7 @@
 // output of the step reads the states of the committed blocks,
 //   out = (w sm_num + phi(q)^T S) / (w sm_den + phi(q)^T Z),
 // and the finished block is then folded in, S += sum_t phi(k_t) v_t^T, Z += sum_t phi(k_t);
-// §3.3 serves both in one kernel launch ("including the causal state update").
+// in §3.3 a single kernel launch does both, the state update included.
 //
 // Each (request, KV head) unit runs the decode step exactly as the decode-only kernel does
 // (the same roles, rings, feature map and shared-normaliser merge; the states are read once,
