@@ -280,6 +280,27 @@ def make_decode_sets(gen, nsets=NSETS, R=R, Hq=HQ, Hkv=HKV, d=D, F=F, B=B, prefi
     return W, cu, sets
 
 
+def host_info():
+    """CPU model, logical core count and the BLAS pool size the float64 oracle runs with."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    blas = None
+    try:
+        import threadpoolctl
+
+        blas = max(i.get("num_threads", 1) for i in threadpoolctl.threadpool_info())
+    except Exception:  # noqa: BLE001
+        pass
+    return {"cpu_model": model, "cpu_count": os.cpu_count(), "blas_threads": blas}
+
+
 def cpu_oracle_decode(budget_s, seed=0):
     """Time the float64 oracle on a bounded sample of the decode-step workload: whole
     requests (all 16 query heads, 32 block tokens) with directly drawn states, one request's
@@ -355,7 +376,7 @@ def bench_reference(args, world, rank):
         "data": "synthetic",
         "config": decode_config(),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, **host_info()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -542,7 +563,7 @@ def bench_decode(args, world, rank, local, gen):
                                 "kind": "oracle",
                                 "sample": f"{n} whole requests of the decode step (16 query heads x "
                                           f"32 tokens, states given; one request repeated), "
-                                          f"{el:.1f} s"}
+                                          f"{el:.1f} s", **host_info()}
     return line
 
 

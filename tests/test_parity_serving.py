@@ -51,7 +51,7 @@ def _commit_prefix(Kp, Vp, W, S, Z, block, lens=None):
 @pytest.mark.parametrize("P", [2048, 8192, 32768])
 def test_prefix_sweep_states_from_long_prefixes(P, block):
     """64 requests whose states are committed from P-token prefixes, 32 tokens per call (the
-    tensor-core commit) or 128 (the CUDA-core commit); the states and the decode step of 2
+    tensor-core commit) or 128 (the CUDA-core commit); the states and the decode step of 8
     sampled requests against the oracle, which builds the states in one shot."""
     R = 64
     gen = torch.Generator(device="cuda")
@@ -69,7 +69,7 @@ def test_prefix_sweep_states_from_long_prefixes(P, block):
     O = bha.hybrid_attn(cu, Q, K, V, S, Z, W, max_block=B)
     torch.cuda.synchronize()
     Wh = host64(W)
-    for r in np.random.default_rng(P).choice(R, 2, replace=False):
+    for r in np.random.default_rng(P).choice(R, 8, replace=False):
         So = np.zeros((1, HKV, F, D))
         Zo = np.zeros((1, HKV, F))
         Kr, Vr = host64(Kp[r]), host64(Vp[r])
@@ -87,7 +87,7 @@ def test_prefix_sweep_states_from_long_prefixes(P, block):
 @pytest.mark.parametrize("P", [8192, 32768])
 def test_prefix_sweep_teacher_long_caches(P):
     """The softmax teacher at 64 requests over caches of P + 32 tokens (at 32K split into key
-    ranges and combined); every row of 2 sampled requests against the oracle."""
+    ranges and combined); every row of 8 sampled requests against the oracle."""
     R, L = 64, P + B
     gen = torch.Generator(device="cuda")
     gen.manual_seed(7 * P)
@@ -100,7 +100,7 @@ def test_prefix_sweep_teacher_long_caches(P):
     # 32K cache is split into key ranges whose partials are combined
     assert (bha.full_prefix_workspace_bytes(R, HQ, HKV, D, B, R * B, L) > 0) == (P == 32768)
     O = host64(bha.full_prefix_attn(cu, kv_len, Q, Kc, Vc, max_block=B))
-    for r in np.random.default_rng(P + 1).choice(R, 2, replace=False):
+    for r in np.random.default_rng(P + 1).choice(R, 8, replace=False):
         sl = slice(B * r, B * r + B)
         want = ref.full_prefix_attn([0, B], [L], host64(Q[sl]), host64(Kc[r:r + 1]), host64(Vc[r:r + 1]))
         assert_close(O[sl], want, TOL_BF16, f"teacher O[{r}] at prefix {P}")
@@ -110,7 +110,7 @@ def test_serving_cycle_ragged_mix_six_layers():
     """128 requests with prefixes uniform on {0, 32, ..., 8192} (committed 128 tokens per call,
     as the serving bench does), 6 layers with independent W, 8 denoising steps of fresh
     activations, a commit of the last step's K/V in every layer, then one more step.  The
-    request with the empty prefix, the one with the longest and two others are checked in
+    request with the empty prefix, the one with the longest and six others are checked in
     every layer at the first and last step and at the step after the commit."""
     R, layers, steps = 128, 6, 8
     plen = inputs.ragged_prefix_lengths(R, seed=5)
@@ -149,7 +149,7 @@ def test_serving_cycle_ragged_mix_six_layers():
 
     order = np.argsort(plen)
     rng = np.random.default_rng(2)
-    reqs = [int(order[0]), int(order[-1])] + [int(r) for r in rng.choice(order[1:-1], 2, replace=False)]
+    reqs = [int(order[0]), int(order[-1])] + [int(r) for r in rng.choice(order[1:-1], 6, replace=False)]
     assert plen[reqs[0]] == 0 and plen[reqs[1]] == Pmax
     for l in range(layers):
         Wh = host64(Ws[l])
