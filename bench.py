@@ -68,6 +68,11 @@ def step_flops(R=R, Hq=HQ, Hkv=HKV, d=D, F=F, B=B):
     return 2 * R * Hq * B * per_q
 
 
+def commit_flops(R=R, Hkv=HKV, d=D, F=F, B=B):
+    """FLOPs of one commit (2 per multiply-add): k.W, phi(k) v^T and the phi sum per token."""
+    return 2 * R * Hkv * B * (d * (F // 2) + F * d + F)
+
+
 def commit_bytes(R=R, Hkv=HKV, d=D, F=F, B=B):
     """S and Z read and written once (fp32), K and V of the block read once, W once."""
     return R * Hkv * (2 * F * d * 4 + 2 * F * 4 + 2 * B * d * 2) + Hkv * d * (F // 2) * 2
@@ -567,9 +572,10 @@ def bench_decode(args, world, rank, local, gen):
     return line
 
 
-def bench_commit(args, world, rank, local, steps):
-    """Block commit for 128 requests x 4 KV heads (d 128, F 256, 32-token blocks): S and Z
-    updated in place; 4 rotating state sets (75 MB each) keep L2 from holding them."""
+def bench_commit(args, world, rank, local, steps, block=B):
+    """Block commit for 128 requests x 4 KV heads (d 128, F 256, `block`-token blocks: 32, the
+    serving shape, or 128, the large-block variant whose contractions are 4x deeper): S and Z
+    updated in place; 4 rotating state sets (75 MB and more each) keep L2 from holding them."""
     from linear_attention_diffusion_hedgehog_b200 import bha
 
     peaks, src = load_peaks()
@@ -577,34 +583,43 @@ def bench_commit(args, world, rank, local, steps):
     gen.manual_seed(99 + rank)
     dev, bf = torch.device("cuda"), torch.bfloat16
     W = (torch.randn((HKV, D, F // 2), generator=gen, device=dev) / D ** 0.5).to(bf)
-    cu = torch.arange(0, (R + 1) * B, B, dtype=torch.int32, device=dev)
-    sets = [dict(K=torch.randn((R * B, HKV, D), generator=gen, device=dev).to(bf),
-                 V=torch.randn((R * B, HKV, D), generator=gen, device=dev).to(bf),
+    cu = torch.arange(0, (R + 1) * block, block, dtype=torch.int32, device=dev)
+    sets = [dict(K=torch.randn((R * block, HKV, D), generator=gen, device=dev).to(bf),
+                 V=torch.randn((R * block, HKV, D), generator=gen, device=dev).to(bf),
                  S=torch.randn((R, HKV, F, D), generator=gen, device=dev),
                  Z=torch.rand((R, HKV, F), generator=gen, device=dev) * 8) for _ in range(NSETS)]
     stream = torch.cuda.Stream()
-    dims = bha.make_dims(R, HKV, HKV, D, F, B, R * B, R, bf)
+    dims = bha.make_dims(R, HKV, HKV, D, F, block, R * block, R, bf)
     variant = bha.kernel_variant(dims, 2)
 
     def step(i):
         s = sets[i % NSETS]
-        bha.commit_block(cu, s["K"], s["V"], W, s["S"], s["Z"], max_block=B, stream=stream)
+        bha.commit_block(cu, s["K"], s["V"], W, s["S"], s["Z"], max_block=block, stream=stream)
 
     ms = max_over_ranks(time_graphed(step, steps, args.warmup, world, stream), world)
     del sets
     torch.cuda.empty_cache()
     ms_step = ms / steps
-    cfg = {"workload": "block commit: fold a 32-token block into S/Z for 128 requests x 4 KV "
+    cfg = {"workload": f"block commit: fold a {block}-token block into S/Z for 128 requests x 4 KV "
                        "heads, head dim 128, feature dim 256", "requests": R, "kv_heads": HKV,
-           "head_dim": D, "feature_dim": F, "block": B,
-           "l2": f"rotating {NSETS} state sets of ~75 MB each, together larger than the 126 MB L2"}
-    return _record("block-commit tokens/s (128 reqs x 4 KV heads)", whole_job_rate(R * B, steps, ms, world),
+           "head_dim": D, "feature_dim": F, "block": block,
+           "l2": f"rotating {NSETS} state sets of ~{commit_bytes(B=block) / 2 / 1e6:.0f} MB each, "
+                 "together larger than the 126 MB L2"}
+    key = "commit" if block == B else f"commit_b{block}"
+    return _record(f"block-commit tokens/s (128 reqs x 4 KV heads, {block}-token blocks)",
+                   whole_job_rate(R * block, steps, ms, world),
                    UNIT, steps, ms_step, cfg, dtype="bf16",
                    precision="bf16 activations; fp32 states and accumulation", kernel_variant=variant,
-                   roofline=_roof(commit_bytes(), ms_step, peaks, src, "commit",
-                                  flops=2 * R * HKV * B * (D * (F // 2) + F * D + F),
-                                  traffic=_traffic_for("commit", variant, "commit_tc.cu")),
+                   roofline=_roof(commit_bytes(B=block), ms_step, peaks, src, "commit",
+                                  flops=commit_flops(B=block),
+                                  traffic=_traffic_for(key, variant, "commit_tc.cu")),
                    gpu_launches=steps)
+
+
+def bench_commit_b128(args, world, rank, local, steps):
+    """The large-block variant of the commit: 128-token blocks (one request per 128-row tile,
+    dS^T contracted over 128 tokens)."""
+    return bench_commit(args, world, rank, local, steps, block=128)
 
 
 def bench_featuremap(args, world, rank, local, steps):
@@ -889,8 +904,8 @@ def bench_per_qhead(args, world, rank, local, steps):
                    gpu_launches=steps)
 
 
-SUB_STEPS = {"commit": 1000, "fused": 1000, "featuremap": 1000, "per_qhead": 1000, "sweep": 500,
-             "cycle": 50}
+SUB_STEPS = {"commit": 1000, "commit_b128": 1000, "fused": 1000, "featuremap": 1000,
+             "per_qhead": 1000, "sweep": 500, "cycle": 50}
 
 
 def main():
@@ -899,8 +914,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["all", "decode", "commit", "fused", "featuremap", "per_qhead",
-                                           "sweep", "cycle"],
+    ap.add_argument("--workload", choices=["all", "decode", "commit", "commit_b128", "fused", "featuremap",
+                                           "per_qhead", "sweep", "cycle"],
                     default="all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -910,8 +925,9 @@ def main():
         bench_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
         return
     world, rank, local = dist_setup(args.gpus)
-    subs = {"commit": bench_commit, "fused": bench_fused, "featuremap": bench_featuremap,
-            "per_qhead": bench_per_qhead, "sweep": bench_sweep, "cycle": bench_cycle}
+    subs = {"commit": bench_commit, "commit_b128": bench_commit_b128, "fused": bench_fused,
+            "featuremap": bench_featuremap, "per_qhead": bench_per_qhead, "sweep": bench_sweep,
+            "cycle": bench_cycle}
     try:
         if args.workload in subs:
             rec = subs[args.workload](args, world, rank, local, args.steps)

@@ -1,18 +1,19 @@
 // Tensor-core block commit for sm_100a (bf16 activations, d = 128, F = 256, blocks of up
-// to 32 tokens).
+// to 128 tokens).
 //
 // Source: "Retrofitting Linear Attention into Diffusion Language Models", §3.1, the commit
 // of a finished block:  S_n = S_{n-1} + sum_{t in B_n} phi(k_t) v_t^T,  Z_n = Z_{n-1} +
 // sum_{t in B_n} phi(k_t),  phi(k) = [softmax(kW), softmax(-kW)].
 //
-// Work unit: four requests that share KV head g (their 4 x 32 key rows form one 128-row
-// MMA tile for u = K W_g).  Per unit:
-//   u     = K W_g                 bf16 MMA, M 128 (4 requests x 32 tokens), N 128, K 128
+// Work unit: 128 / kBt requests that share KV head g, kBt = 32, 64 or 128 the smallest that
+// holds the call's largest block (their key rows form one 128-row MMA tile for u = K W_g).
+// Per unit:
+//   u     = K W_g                 bf16 MMA, M 128 (requests x kBt tokens), N 128, K 128
 //   phi   = [softmax(u), softmax(-u)] per row on CUDA cores (two threads per row), rounded
 //           to bf16 into shared memory as the B operand of the next MMA; rows past a
 //           request's block are zero, so they add nothing
 //   dZ    = column sums of the bf16 phi over each request's tokens (CUDA cores)
-//   dS^T  = V_r^T phi_r           bf16 MMA per request, M 128 (d), N 256 (F), K 32 (tokens)
+//   dS^T  = V_r^T phi_r           bf16 MMA per request, M 128 (d), N 256 (F), K kBt (tokens)
 //                                 into one of two TMEM buffers
 //   S += dS, Z += dZ               TMA bulk reduce-add: each of 8 warps copies 16 columns of
 //                                 dS^T at a time from TMEM (its lane quarter = 32 values of d)
@@ -38,15 +39,11 @@ namespace {
 constexpr int kD = 128;
 constexpr int kF = 256;
 constexpr int kFh = 128;
-constexpr int kBlk = 32;
-constexpr int kReq = 4;          // requests per unit
-constexpr int kM = kReq * kBlk;  // 128 key rows
+constexpr int kM = 128;          // key rows per unit: kM / kBt requests of up to kBt tokens
 constexpr int kThreads = 320;
 
 constexpr uint32_t kKBytes = kM * kD * 2;        // 32 KiB: [d half][128 rows][128 B]
 constexpr uint32_t kWBytes = kD * kFh * 2;       // 32 KiB: [f half][128 rows of d][128 B]
-constexpr uint32_t kVReqBytes = kBlk * kD * 2;   // 8 KiB per request: [d half][32 rows][128 B]
-constexpr uint32_t kPhiReqBytes = kBlk * kF * 2; // 16 KiB per request: [f quarter][32 rows][128 B]
 constexpr int kRedRows = 16;                      // F rows per reduce-add tile
 
 constexpr uint32_t kColU = 0;     // u (128 columns), inside dS buffer 0
@@ -57,25 +54,38 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kIdKW = tc::instr_desc(1, 0, 1, kM, kFh);   // A K-major, B MN-major
 constexpr uint32_t kIdVP = tc::instr_desc(1, 1, 1, kD, kF);    // A MN-major (V^T), B MN-major
 
+// Block rows per request kBt = 32, 64 or 128 (the smallest that holds the call's largest
+// block); a unit is kM / kBt requests.  Per request, V is [d half][kBt rows][128 B] and phi
+// [F quarter][kBt rows][128 B], so the buffers of a unit have the same size for every kBt.
+template <int kBt>
+struct Shape {
+  static constexpr int kReq = kM / kBt;
+  static constexpr uint32_t kVReqBytes = kBt * kD * 2;
+  static constexpr uint32_t kPhiReqBytes = kBt * kF * 2;
+};
+
+template <int kBt>
 struct __align__(1024) Smem {
   uint8_t k[kKBytes];
   uint8_t w[kWBytes];
-  uint8_t v[kReq][kVReqBytes];
-  uint8_t phi[kReq][kPhiReqBytes];
-  float dz[kReq][kF];
+  uint8_t v[Shape<kBt>::kReq][Shape<kBt>::kVReqBytes];
+  uint8_t phi[Shape<kBt>::kReq][Shape<kBt>::kPhiReqBytes];
+  float dz[Shape<kBt>::kReq][kF];
   float red[8][2][kRedRows * 32];  // per update warp, double-buffered: [16 rows of F][32 d]
   uint64_t k_full, k_empty, v_full, v_empty, w_full, u_full, phi_ready;
   uint64_t d_full[2], d_empty[2], drain;
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory budget");
+static_assert(sizeof(Smem<32>) + 1024 <= 232448 && sizeof(Smem<128>) + 1024 <= 232448,
+              "shared memory budget");
 
 struct Req {
   int lo, n, slot;  // n = 0: absent (no request, empty block or invalid)
 };
 
-// The four requests of unit (j0, g); every role decodes them identically.
+// The kReq requests of unit (j0, g); every role decodes them identically.
+template <int kReq>
 __device__ __forceinline__ void decode_unit(const TcCommitParams& p, int j0, bool report,
                                             Req (&rq)[kReq]) {
 #pragma unroll
@@ -95,9 +105,13 @@ __device__ __forceinline__ void decode_unit(const TcCommitParams& p, int j0, boo
   }
 }
 
+template <int kBt>
 __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_constant__ TcCommitParams p) {
+  constexpr int kReq = Shape<kBt>::kReq;
+  constexpr uint32_t kVReqBytes = Shape<kBt>::kVReqBytes;
+  constexpr uint32_t kPhiReqBytes = Shape<kBt>::kPhiReqBytes;
   extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<kBt>& sm = *reinterpret_cast<Smem<kBt>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &sm.abort_flag;
   const long long lim = p.wait_limit;
@@ -160,12 +174,12 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
           g_res = g;
         }
         if (k >= 1 && !tc::mbar_wait(&sm.k_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
-        tc::mbar_arrive_expect_tx(&sm.k_full, nreq * 2 * (kBlk * 64 * 2));
+        tc::mbar_arrive_expect_tx(&sm.k_full, nreq * 2 * (kBt * 64 * 2));
 #pragma unroll
         for (int j = 0; j < kReq; ++j) {
           if (rq[j].n == 0) continue;
-          tc::tma_load_3d(sm.k + j * kBlk * 128, &p.tm_k, &sm.k_full, 0, g, rq[j].lo);
-          tc::tma_load_3d(sm.k + kKBytes / 2 + j * kBlk * 128, &p.tm_k, &sm.k_full, 64, g, rq[j].lo);
+          tc::tma_load_3d(sm.k + j * kBt * 128, &p.tm_k, &sm.k_full, 0, g, rq[j].lo);
+          tc::tma_load_3d(sm.k + kKBytes / 2 + j * kBt * 128, &p.tm_k, &sm.k_full, 64, g, rq[j].lo);
         }
         armed_k = k & 1;
         if (k >= 1 && !tc::mbar_wait(&sm.v_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
@@ -227,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
           tc::tc_fence_after();
           const uint32_t va = tc::smem_u32(sm.v[j]), pa = tc::smem_u32(sm.phi[j]);
 #pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk) {
+          for (int kk = 0; kk < kBt / 16; ++kk) {
             // A = V^T (M = d, K = tokens), MN-major: d halves 4 KiB apart, 8-token groups 1 KiB
             const uint64_t a = tc::smem_desc(va + kk * 2048, kVReqBytes / 2, 1024, tc::kSwizzle128B);
             // B = phi (K = tokens, N = F), MN-major: F quarters 4 KiB apart
@@ -254,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
     const int half = sw >> 2;         // feature-map half / F half of the state update
     const float sgn = half ? -1.f : 1.f;
     const int wq = warp & 3;          // TMEM lane quarter
-    const int row = wq * 32 + lane;   // key row = 32 j + t during the feature map; d afterwards
+    const int row = wq * 32 + lane;   // key row = kBt j + t during the feature map; d afterwards
     const int tid = sw * 32 + lane;   // 0..255
     const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
     const float log2e = 1.4426950408889634f;
@@ -276,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
       good = tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim) && good;
       tc::tc_fence_after();
       // ---- this thread's half of phi for key row `row`, rounded to bf16
-      const int jr = row >> 5, t = row & 31;
+      const int jr = row / kBt, t = row % kBt;
       const bool live = t < rq[jr].n;
       float e[kFh];
       {
@@ -320,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
 #pragma unroll
       for (int j = 0; j < kReq; ++j) {
         const int n = rq[j].n;
-        if (n >= kBlk || n == 0) continue;
-        const int per_half = (kBlk - n) * 8;
+        if (n >= kBt || n == 0) continue;
+        const int per_half = (kBt - n) * 8;
         for (int i = tid; i < 2 * per_half; i += 256) {
           const int hh = i / per_half, rem = i % per_half;
           *reinterpret_cast<uint4*>(sm.v[j] + hh * (kVReqBytes / 2) + (n + rem / 8) * 128 + (rem % 8) * 16) =
@@ -404,17 +418,21 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
 }  // namespace
 
 bool commit_tc_supports(const CommitArgs& a, bool act_bf16) {
-  return act_bf16 && a.d == kD && a.F == kF && a.Bmax <= kBlk &&
+  return act_bf16 && a.d == kD && a.F == kF && a.Bmax <= kM &&
          (long long)a.num_slots * a.Hkv * kF * kD < (1ll << 40);
 }
 
-cudaError_t launch_commit_tc(const CommitArgs& a, cudaStream_t st) {
+namespace {
+
+template <int kBt>
+cudaError_t launch_commit_tc_bt(const CommitArgs& a, cudaStream_t st) {
+  constexpr int kReq = Shape<kBt>::kReq;
   TcCommitParams p;
   const uint64_t T = (uint64_t)a.T;
   {
     const uint64_t dims[3] = {kD, (uint64_t)a.Hkv, T};
     const uint64_t strides[2] = {kD * 2, (uint64_t)a.Hkv * kD * 2};
-    const uint32_t box[3] = {64, 1, kBlk};
+    const uint32_t box[3] = {64, 1, kBt};
     if (!make_tensor_map(&p.tm_k, false, 3, a.K, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
     if (!make_tensor_map(&p.tm_v, false, 3, a.V, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
   }
@@ -448,11 +466,20 @@ cudaError_t launch_commit_tc(const CommitArgs& a, cudaStream_t st) {
   int grid = nsm;
   if (a.Hkv <= nsm) grid = (nsm / a.Hkv) * a.Hkv;
   if (grid > units) grid = units;
-  const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(commit_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = sizeof(Smem<kBt>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(commit_tc_kernel<kBt>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  commit_tc_kernel<<<grid, kThreads, smem, st>>>(p);
+  commit_tc_kernel<kBt><<<grid, kThreads, smem, st>>>(p);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+// Requests of up to 32, 64 or 128 tokens per unit tile: 4, 2 or 1 request per unit.
+cudaError_t launch_commit_tc(const CommitArgs& a, cudaStream_t st) {
+  if (a.Bmax <= 32) return launch_commit_tc_bt<32>(a, st);
+  if (a.Bmax <= 64) return launch_commit_tc_bt<64>(a, st);
+  return launch_commit_tc_bt<128>(a, st);
 }
 
 }  // namespace bha

@@ -38,6 +38,18 @@ def test_commit_bytes():
     assert b.commit_bytes() == rmw + kv + Hkv * d * (F // 2) * 2 == 143_785_984
 
 
+def test_large_block_commit_bytes_and_flops():
+    """128-token blocks: four times the K/V bytes of the serving commit, the same state
+    traffic; per token k.W (d x F/2), phi(k) v^T (F x d) and the phi sum (F)."""
+    b = _bench()
+    R, Hkv, d, F, B = 128, 4, 128, 256, 128
+    rmw = 2 * (R * Hkv * F * d * 4 + R * Hkv * F * 4)
+    kv = 2 * R * B * Hkv * d * 2
+    assert b.commit_bytes(B=B) == rmw + kv + Hkv * d * (F // 2) * 2 == 168_951_808
+    assert b.commit_flops(B=B) == 2 * R * Hkv * B * (d * F // 2 + F * d + F) == 6_476_005_376
+    assert b.commit_flops() * 4 == b.commit_flops(B=B)
+
+
 def test_teacher_bytes_over_the_prefix_sweep():
     b = _bench()
     for P, want in ((512, 88_080_384), (2048, 289_406_976), (8192, 1_094_713_344),

@@ -305,6 +305,52 @@ def test_commit_ragged_with_slots_and_empty_blocks():
     np.testing.assert_array_equal(host64(S[1]), S_np[1])   # no request: untouched
 
 
+@pytest.mark.parametrize("bmax,lens", [
+    (64, [64, 0, 1, 63, 40, 64, 17]),          # two requests per tile
+    (48, [48, 3, 0, 47, 48]),                  # rounded up to 64-row request slots
+    (128, [128, 0, 1, 127, 100, 128, 65]),     # one request per tile
+    (128, [100]),                              # one request, fewer tokens than the tile
+])
+def test_commit_large_blocks_tensor_core(bmax, lens):
+    """Blocks of up to 64 or 128 tokens on the tensor-core commit (64- or 128-row request
+    slots, so 2 or 1 requests per 128-row tile): ragged lengths including empty blocks, a
+    permuted slot map and random initial states, against the oracle's commit."""
+    R = len(lens)
+    c = inputs.decode_case(R=R, Hq=4, Hkv=4, d=128, F=256, block_lens=lens, prefix_lens=0,
+                           seed=60 + bmax + R, dtype="bf16")
+    dims = bha.make_dims(R, 4, 4, 128, 256, bmax, int(c.cu_blk[-1]), R + 2, torch.bfloat16)
+    assert bha.kernel_variant(dims, 2) == 1
+    S_np, Z_np = inputs.random_states(R + 2, 4, 256, 128, prefix_len=256, seed=bmax)
+    slots = np.random.default_rng(bmax + R).permutation(R + 2)[:R].astype(np.int32)
+    S, Z = dev(S_np, torch.float32), dev(Z_np, torch.float32)
+    cu = torch.tensor(c.cu_blk, dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bha.commit_block(cu, dev(c.K, torch.bfloat16), dev(c.V, torch.bfloat16),
+                     dev(c.W, torch.bfloat16), S, Z, max_block=bmax,
+                     state_slot=torch.tensor(slots, device="cuda"), dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    So, Zo = ref.commit_block(c.cu_blk, c.K, c.V, c.W, S_np, Z_np, slots)
+    assert_close(host64(S), So, TOL_BF16, "S")
+    assert_close(host64(Z), Zo, TOL_BF16, "Z")
+    for sl in set(range(R + 2)) - {int(slots[r]) for r in range(R) if lens[r] > 0}:
+        np.testing.assert_array_equal(host64(S[sl]), S_np[sl])   # no token committed there
+
+
+def test_commit_128_token_blocks_128_requests_one_shot():
+    """128 requests x 4 KV heads folding 1024-token prefixes into zero states in 8 commits of
+    128-token blocks (the large-block commit at full width); every request against the
+    oracle's one-shot build."""
+    c = inputs.decode_case(R=128, Hq=4, Hkv=4, d=128, F=256, block_lens=32, prefix_lens=1024,
+                           seed=61, dtype="bf16")
+    dims = bha.make_dims(128, 4, 4, 128, 256, 128, 128 * 128, 128, torch.bfloat16)
+    assert bha.kernel_variant(dims, 2) == 1
+    S, Z = build_states_on_gpu(c, block=128)
+    So, Zo = oracle_states(c)
+    assert_close(host64(S), So, TOL_BF16, "S after 8 commits of 128 tokens")
+    assert_close(host64(Z), Zo, TOL_BF16, "Z after 8 commits of 128 tokens")
+
+
 # ------------------------------------------------------------------- generic dims
 
 def test_generic_max_dims_fp32():

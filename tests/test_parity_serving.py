@@ -50,9 +50,10 @@ def _commit_prefix(Kp, Vp, W, S, Z, block, lens=None):
 @pytest.mark.parametrize("block", [32, 128])
 @pytest.mark.parametrize("P", [2048, 8192, 32768])
 def test_prefix_sweep_states_from_long_prefixes(P, block):
-    """64 requests whose states are committed from P-token prefixes, 32 tokens per call (the
-    tensor-core commit) or 128 (the CUDA-core commit); the states and the decode step of 8
-    sampled requests against the oracle, which builds the states in one shot."""
+    """64 requests whose states are committed from P-token prefixes, 32 tokens per call (four
+    requests per 128-row tile of the tensor-core commit) or 128 (one request per tile); the
+    states and the decode step of 8 sampled requests against the oracle, which builds the
+    states in one shot."""
     R = 64
     gen = torch.Generator(device="cuda")
     gen.manual_seed(P + block)
