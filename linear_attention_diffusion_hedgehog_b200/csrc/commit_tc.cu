@@ -22,12 +22,17 @@
 //                                 L2; Z by reducing atomic adds.  No thread waits on a load of
 //                                 S, and the other dS buffer's MMA overlaps the update.
 // Computing dS transposed (lanes = d) is what lets each warp write whole 128-byte rows of its
-// shared tile, one per instruction, without bank conflicts.
+// shared tile, one per instruction, without bank conflicts.  When each CTA has one unit, its
+// states are prefetched into L2 as soon as K, V and W have landed, so the reduce-adds find
+// them there.
 //
 // Roles (320 threads): warp 0 TMA producer (K, V, W), warp 1 TMEM owner and MMA issuer,
 // warps 2-9 feature map, dZ and the state update.  Every wait is bounded; on expiry the CTA
 // records BHA_ERR_TIMEOUT, drains its copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
+#include <cuda_fp16.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -103,6 +108,116 @@ __device__ __forceinline__ void decode_unit(const TcCommitParams& p, int j0, boo
     rq[j].n = rr.n;
     rq[j].slot = slot;
   }
+}
+
+// One thread's half of phi for one key row: e = 2^{(s u - max_f s u) log2 e} over the 128
+// values s u of its half (s = +1 or -1, u read from TMEM a 32-column chunk at a time),
+// phi = e / sum e rounded to bf16 and written as 16 row chunks of 16 bytes, chunk c of F
+// quarter q at quarter q, chunk position c ^ (t % 8) (the 128-byte swizzle the MMA reads).
+// Rows past the block (live false) are written as zeros, selected rather than multiplied, so
+// stale shared memory cannot inject a NaN.
+//
+// Two forms with the same result up to rounding: phi_row_fp32 keeps the 128 e values in fp32
+// registers; phi_row_fp16 reads u twice and keeps e as fp16 pairs (11 significant bits,
+// eight times finer than the bf16 phi they become; e <= 1 and the values fp16 flushes are
+// below 2^-24 of the sum), which leaves about 64 more registers for the rest of the thread.
+__device__ __forceinline__ void phi_row_store(uint8_t* row_base, uint32_t quarter_bytes, int t, bool live,
+                                              int c, uint4 v) {
+  const int quarter = c >> 3, ch = c & 7;
+  *reinterpret_cast<uint4*>(row_base + quarter * quarter_bytes + ((ch ^ (t & 7)) << 4)) =
+      live ? v : make_uint4(0, 0, 0, 0);
+}
+
+__device__ __forceinline__ void phi_row_fp32(uint32_t tu, float sgn, uint8_t* row_base,
+                                             uint32_t quarter_bytes, int t, bool live) {
+  const float log2e = 1.4426950408889634f;
+  float e[kFh];
+  float ext = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < kFh / 32; ++c) {
+    float uv[32];
+    tc::tmem_ld32(tu + c * 32, uv);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      e[c * 32 + i] = sgn * uv[i];
+      ext = fmaxf(ext, e[c * 32 + i]);
+    }
+  }
+  float esum = 0.f;
+#pragma unroll
+  for (int i = 0; i < kFh; ++i) {
+    e[i] = tc::ex2((e[i] - ext) * log2e);
+    esum += e[i];
+  }
+  const float inv = 1.f / esum;
+#pragma unroll
+  for (int c = 0; c < kFh / 8; ++c)
+    phi_row_store(row_base, quarter_bytes, t, live, c,
+                  make_uint4(pack_bf16(e[8 * c] * inv, e[8 * c + 1] * inv),
+                             pack_bf16(e[8 * c + 2] * inv, e[8 * c + 3] * inv),
+                             pack_bf16(e[8 * c + 4] * inv, e[8 * c + 5] * inv),
+                             pack_bf16(e[8 * c + 6] * inv, e[8 * c + 7] * inv)));
+}
+
+__device__ __forceinline__ void phi_row_fp16(uint32_t tu, float sgn, uint8_t* row_base,
+                                             uint32_t quarter_bytes, int t, bool live) {
+  const float log2e = 1.4426950408889634f;
+  float ext = -INFINITY;
+#pragma unroll 1
+  for (int c = 0; c < kFh / 32; ++c) {
+    float uv[32];
+    tc::tmem_ld32(tu + c * 32, uv);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ext = fmaxf(ext, sgn * uv[i]);
+  }
+  float esum = 0.f;
+  __half2 eh[kFh / 2];
+#pragma unroll
+  for (int c = 0; c < kFh / 32; ++c) {
+    float uv[32];
+    tc::tmem_ld32(tu + c * 32, uv);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const float e0 = tc::ex2((sgn * uv[i] - ext) * log2e);
+      const float e1 = tc::ex2((sgn * uv[i + 1] - ext) * log2e);
+      esum += e0 + e1;
+      eh[(c * 32 + i) / 2] = __floats2half2_rn(e0, e1);
+    }
+  }
+  const float inv = 1.f / esum;
+#pragma unroll
+  for (int c = 0; c < kFh / 8; ++c) {
+    const float2 p0 = __half22float2(eh[4 * c]), p1 = __half22float2(eh[4 * c + 1]);
+    const float2 p2 = __half22float2(eh[4 * c + 2]), p3 = __half22float2(eh[4 * c + 3]);
+    phi_row_store(row_base, quarter_bytes, t, live, c,
+                  make_uint4(pack_bf16(p0.x * inv, p0.y * inv), pack_bf16(p1.x * inv, p1.y * inv),
+                             pack_bf16(p2.x * inv, p2.y * inv), pack_bf16(p3.x * inv, p3.y * inv)));
+  }
+}
+
+// dZ[f] of one request: the sum over its n tokens of the bf16 phi column f (base: the
+// request's phi at f's quarter and f's 2-byte position in its chunk ch); kAcc independent
+// partial sums keep that many loads in flight.
+template <int kAcc>
+__device__ __forceinline__ float phi_column_sum(const uint8_t* base, int n, int ch) {
+  auto at = [&](int tt) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + tt * 128 + ((ch ^ (tt & 7)) << 4)));
+  };
+  float a[kAcc];
+#pragma unroll
+  for (int i = 0; i < kAcc; ++i) a[i] = 0.f;
+  int tt = 0;
+  for (; tt + kAcc <= n; tt += kAcc)
+#pragma unroll
+    for (int i = 0; i < kAcc; ++i) a[i] += at(tt + i);
+  for (; tt < n; ++tt) a[0] += at(tt);
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < kAcc; ++i) sum += a[i];
+  return sum;
 }
 
 template <int kBt>
@@ -191,6 +306,26 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
           tc::tma_load_3d(sm.v[j] + kVReqBytes / 2, &p.tm_v, &sm.v_full, 64, g, rq[j].lo);
         }
         armed_v = k & 1;
+        // When every CTA has a single unit (the serving commit: 128 requests x 4 KV heads in
+        // 128 units), the unit's states are asked into L2 once its K, V and W have landed:
+        // their HBM reads then overlap the feature map instead of starting with the first
+        // reduce-add, and do not delay the loads the feature map needs first (30.9 us
+        // against 34.5 us without the prefetch and 32.2 us issuing it with K and V).  With
+        // more units per CTA one unit's state traffic already overlaps the next unit's
+        // compute, and the extra requests only contend.
+        if (units <= (int)gridDim.x) {
+          if (!tc::mbar_wait(&sm.k_full, k & 1, abort_flag, lim) || !tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim) ||
+              !tc::mbar_wait(&sm.w_full, (w_loads - 1) & 1, abort_flag, lim)) { ok = false; break; }
+#pragma unroll 1
+          for (int j = 0; j < kReq; ++j) {
+            if (rq[j].n == 0) continue;
+            // one (slot, head) state: 128 KiB, asked for in four 32 KiB pieces
+            constexpr uint32_t kPiece = kF * kD * 4 / 4;
+            const char* sb = reinterpret_cast<const char*>(p.S + ((size_t)rq[j].slot * p.Hkv + g) * kF * kD);
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) tc::bulk_prefetch_l2(sb + c * kPiece, kPiece);
+          }
+        }
         ++k;
       }
       volatile int never = 0;
@@ -271,7 +406,6 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
     const int row = wq * 32 + lane;   // key row = kBt j + t during the feature map; d afterwards
     const int tid = sw * 32 + lane;   // 0..255
     const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
-    const float log2e = 1.4426950408889634f;
     int k = 0, rc = 0, nred = 0;
     // A failed wait does not leave the loop at once: these 256 threads meet at a named barrier
     // each unit, so all of them reach it and leave together, decided by the reducing barrier.
@@ -289,45 +423,17 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
       good = tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim) && good;
       good = tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim) && good;
       tc::tc_fence_after();
-      // ---- this thread's half of phi for key row `row`, rounded to bf16
-      const int jr = row / kBt, t = row % kBt;
-      const bool live = t < rq[jr].n;
-      float e[kFh];
+      // ---- this thread's half of phi for key row `row`, rounded to bf16.  With 32-row request
+      // slots the fp32 form fits the register budget; the 64- and 128-row instantiations
+      // spill with it (about 200 bytes) and take the fp16 form.
       {
-        float ext = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < kFh / 32; ++c) {
-          float uv[32];
-          tc::tmem_ld32(tl + kColU + c * 32, uv);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            e[c * 32 + i] = sgn * uv[i];
-            ext = fmaxf(ext, e[c * 32 + i]);
-          }
-        }
-        float esum = 0.f;
-#pragma unroll
-        for (int i = 0; i < kFh; ++i) {
-          e[i] = tc::ex2((e[i] - ext) * log2e);
-          esum += e[i];
-        }
-        const float inv = 1.f / esum;
-        // phi_j as the B operand: F quarter a = 2 half + f / 64, row t, 16-byte chunk
-        // (f % 64) / 8 stored at chunk ^ (t % 8).  Rows past the block are written as zeros
-        // (selected, not multiplied, so stale shared memory cannot inject a NaN).
-        uint8_t* base = sm.phi[jr] + (2 * half) * (kPhiReqBytes / 4) + t * 128;
-#pragma unroll
-        for (int c = 0; c < kFh / 8; ++c) {
-          uint4 v4 = make_uint4(0, 0, 0, 0);
-          if (live)
-            v4 = make_uint4(pack_bf16(e[8 * c] * inv, e[8 * c + 1] * inv),
-                            pack_bf16(e[8 * c + 2] * inv, e[8 * c + 3] * inv),
-                            pack_bf16(e[8 * c + 4] * inv, e[8 * c + 5] * inv),
-                            pack_bf16(e[8 * c + 6] * inv, e[8 * c + 7] * inv));
-          const int quarter = c >> 3, ch = c & 7;
-          *reinterpret_cast<uint4*>(base + quarter * (kPhiReqBytes / 4) + ((ch ^ (t & 7)) << 4)) = v4;
-        }
+        const int jr = row / kBt, t = row % kBt;
+        const bool live = t < rq[jr].n;
+        uint8_t* row_base = sm.phi[jr] + (2 * half) * (kPhiReqBytes / 4) + t * 128;
+        if constexpr (kBt == 32)
+          phi_row_fp32(tl + kColU, sgn, row_base, kPhiReqBytes / 4, t, live);
+        else
+          phi_row_fp16(tl + kColU, sgn, row_base, kPhiReqBytes / 4, t, live);
       }
       // rows of V past a request's block (or of an absent request) are cleared, so that
       // nothing from another request can leak in through 0 x (non-finite) products
@@ -342,30 +448,42 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
               make_uint4(0, 0, 0, 0);
         }
       }
-      tc::tc_fence_before();
-      if (tc::named_barrier_any(1, 256, !good)) break;
-      tc::tc_fence_after();
-      // ---- dZ[j][f] = sum over the block's tokens of the bf16 phi (thread tid owns f = tid)
-      {
-        const int f = tid, quarter = f >> 6, ch = (f & 63) >> 3, w8 = f & 7;
-#pragma unroll
-        for (int j = 0; j < kReq; ++j) {
-          float acc = 0.f;
-          if (rq[j].n > 0) {
-            const uint8_t* base = sm.phi[j] + quarter * (kPhiReqBytes / 4);
-            for (int tt = 0; tt < rq[j].n; ++tt) {
-              const __nv_bfloat16 vb =
-                  *reinterpret_cast<const __nv_bfloat16*>(base + tt * 128 + ((ch ^ (tt & 7)) << 4) + w8 * 2);
-              acc += __bfloat162float(vb);
-            }
-          }
-          sm.dz[j][f] = acc;
-        }
-      }
+      // phi and the cleared V rows go to the tensor cores (async proxy); once all 256 threads
+      // have written theirs, the dS^T products may start
       tc::fence_proxy_async_smem();
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sm.phi_ready);
+      // ---- dZ[j][f] = sum over the block's tokens of the bf16 phi (thread tid owns f = tid).
+      // With four requests per tile it is summed before phi is handed to the dS^T products
+      // (one running sum: the register budget has no room for more); with one or two it is
+      // summed while the first product runs, four partial sums at a time.  (Both measured:
+      // 30.9 us and 41.7 us at 32- and 128-token blocks, against 31.8 and 52.1 us the other
+      // way round.)
+      const int zf = tid, zq = zf >> 6, zch = (zf & 63) >> 3, zw = zf & 7;
+      auto column_sums = [&](auto acc_tag) {
+        constexpr int kAcc = decltype(acc_tag)::value;
+#pragma unroll 1
+        for (int j = 0; j < kReq; ++j)
+          sm.dz[j][zf] = phi_column_sum<kAcc>(sm.phi[j] + zq * (kPhiReqBytes / 4) + zw * 2, rq[j].n, zch);
+      };
+      if constexpr (kBt == 32) {
+        tc::tc_fence_before();
+        if (tc::named_barrier_any(1, 256, !good)) break;
+        tc::tc_fence_after();
+        column_sums(std::integral_constant<int, 1>{});
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&sm.phi_ready);
+      } else {
+        // phi and the cleared V rows go to the tensor cores (async proxy) once all 256 threads
+        // have written theirs
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        if (tc::named_barrier_any(1, 256, !good)) break;
+        tc::tc_fence_after();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&sm.phi_ready);
+        column_sums(std::integral_constant<int, 4>{});
+      }
 
       // ---- state update per request: S[f][d] += dS^T[d][f] by tiled reduce-add, Z[f] += dZ[f]
       for (int j = 0; j < kReq; ++j) {
