@@ -112,7 +112,9 @@ int bha_hybrid_attn_commit(const bha_dims* dims, const int32_t* cu_blk, const in
 /* Block commit (§3.1: S_n = S_{n-1} + sum_{t in B_n} phi(k_t) v_t^T, Z_n likewise), in place.
  *   K/V [T][Hkv][d] activation dtype, W [Hkv][d][F/2]; S, Z updated in place (fp32).
  * Any b_r >= 0 is allowed (b_r = 0 leaves the slot untouched).  Two requests must not
- * name the same slot in one call. */
+ * name the same slot in one call.  bf16 with d = 128 and F = 256 runs on the tensor-core
+ * kernel for every max_block up to 128 (its 128-row tiles hold 4, 2 or 1 requests of up to
+ * 32, 64 or 128 tokens). */
 int bha_commit_block(const bha_dims* dims, const int32_t* cu_blk, const int32_t* state_slot,
                      const void* K, const void* V, const void* W, float* S, float* Z,
                      int32_t* dev_err, void* stream);
