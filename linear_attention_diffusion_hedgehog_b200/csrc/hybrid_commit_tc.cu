@@ -15,10 +15,14 @@
 //                                  ring stage the unit's last state group has released; the
 //                                  other rows are ignored), N 128, into the feature-map
 //                                  columns the unit has finished with
-//   phi  = [softmax(u_k), softmax(-u_k)] per block row, 8 rows per feature-map warp,
-//          rounded to bf16 into that same stage (the producer holds it back until dS^T and
-//          dZ have read it); rows past the block are zero
-//   dZ   = column sums of the bf16 phi, added to Z with reducing atomics
+//   phi  = [softmax(u_k), softmax(-u_k)] per block row: the feature-map warps stage u_k's 32
+//          rows in the stage's second half (fp32), then all eight feature-map and epilogue
+//          warps (idle between the unit's output and its dS^T) form phi, eight threads per row
+//          agreeing on its max, min and sums by shuffles, rounded to bf16 into the stage's
+//          first half (the producer holds the stage back until dS^T and dZ have read it);
+//          rows past the block are zero
+//   dZ   = column sums of the bf16 phi (one column per thread of the eight warps), added to
+//          Z with reducing atomics
 //   dS^T = V^T phi                 bf16 MMA, M 128 (d), N 256 (F), K 32, into the accumulator
 //                                  columns once the epilogue has read the output
 //   S   += dS                      the epilogue warps add dS^T into S with reducing atomics
@@ -88,7 +92,7 @@ struct __align__(1024) Smem {
   uint64_t s_full[kStages], s_empty[kStages];
   uint64_t e_ready[kGroups], p_ready;
   uint64_t w_full, u_full, acc_full, acc_empty, drain, fin_full[2], fin_empty[2];
-  uint64_t pv_done, kc_full, uk_done, phi_ready, ds_full, ds_empty, commit_done;
+  uint64_t pv_done, kc_full, uk_done, u_staged, phi_ready, ds_full, ds_empty, commit_done;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -127,6 +131,81 @@ __device__ __forceinline__ bool next_unit(const TcHybridParams& p, int units, in
   return false;
 }
 
+// phi of the block's rows from u_k staged in shared memory (U: [32 rows][128] fp32), by the
+// eight feature-map and epilogue warps: thread gt (0..255) owns row gt / 8 and u columns
+// 16 (gt % 8) .. + 15, so the eight lanes of a row agree on its max, min and sums by
+// shuffles.  phi = [e+ / sum e+, e- / sum e-] rounded to bf16 into phib as the B operand of
+// dS^T: F quarter a = f / 64, row t, 16-byte chunk (f % 64) / 8 stored at chunk ^ (t % 8);
+// rows past the block (t >= n) are written as zeros.
+__device__ __forceinline__ void block_phi(const float* U, uint8_t* phib, int gt, int n) {
+  const float log2e = 1.4426950408889634f;
+  const int t = gt >> 3, s8 = gt & 7;
+  float u[16];
+  const float4* src = reinterpret_cast<const float4*>(U + t * kFh + 16 * s8);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float4 v = src[i];
+    u[4 * i] = v.x;
+    u[4 * i + 1] = v.y;
+    u[4 * i + 2] = v.z;
+    u[4 * i + 3] = v.w;
+  }
+  float mx = u[0], mn = u[0];
+#pragma unroll
+  for (int i = 1; i < 16; ++i) {
+    mx = fmaxf(mx, u[i]);
+    mn = fminf(mn, u[i]);
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  const float bx = mx * log2e, bn = mn * log2e;
+  float ep[16], em[16], sp = 0.f, sm_ = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float a = u[i] * log2e;
+    ep[i] = tc::ex2(a - bx);
+    em[i] = tc::ex2(bn - a);
+    sp += ep[i];
+    sm_ += em[i];
+  }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    sp += __shfl_xor_sync(0xffffffffu, sp, o);
+    sm_ += __shfl_xor_sync(0xffffffffu, sm_, o);
+  }
+  const bool live = t < n;
+  const float ip = 1.f / sp, im = 1.f / sm_;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float* e = h ? em : ep;
+    const float sc = h ? im : ip;
+    // features h F/2 + 16 s8 + i: F quarter 2 h + s8 / 4, chunks 2 (s8 % 4) and 2 (s8 % 4) + 1
+    uint8_t* rowp = phib + (2 * h + (s8 >> 2)) * (kPhiBytes / 4) + t * 128;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int ch = 2 * (s8 & 3) + q;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (live)
+        v = make_uint4(pack_bf16(e[8 * q] * sc, e[8 * q + 1] * sc), pack_bf16(e[8 * q + 2] * sc, e[8 * q + 3] * sc),
+                       pack_bf16(e[8 * q + 4] * sc, e[8 * q + 5] * sc), pack_bf16(e[8 * q + 6] * sc, e[8 * q + 7] * sc));
+      *reinterpret_cast<uint4*>(rowp + ((ch ^ (t & 7)) << 4)) = v;
+    }
+  }
+}
+
+// dZ[f]: the column sum of the bf16 phi over the block's n rows.
+__device__ __forceinline__ float block_dz(const uint8_t* phib, int f, int n) {
+  const int quarter = f >> 6, ch = (f & 63) >> 3, w8 = f & 7;
+  const uint8_t* base = phib + quarter * (kPhiBytes / 4) + w8 * 2;
+  float acc = 0.f;
+  for (int tt = 0; tt < n; ++tt)
+    acc += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + tt * 128 + ((ch ^ (tt & 7)) << 4)));
+  return acc;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __grid_constant__ TcHybridCommitParams pc) {
   const TcHybridParams& p = pc.h;
   extern __shared__ uint8_t smem_raw[];
@@ -162,10 +241,11 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
     tc::mbar_init(&sm.pv_done, 1);
     tc::mbar_init(&sm.kc_full, 1);
     tc::mbar_init(&sm.uk_done, 1);
-    tc::mbar_init(&sm.phi_ready, 4);    // the four feature-map warps, 8 block rows each
+    tc::mbar_init(&sm.u_staged, 4);     // the four feature-map warps, 8 block rows each
+    tc::mbar_init(&sm.phi_ready, 8);    // the feature-map and epilogue warps, 4 block rows each
     tc::mbar_init(&sm.ds_full, 1);
     tc::mbar_init(&sm.ds_empty, 4);     // the four epilogue warps
-    tc::mbar_init(&sm.commit_done, 4);  // the feature-map warps, done reading phi
+    tc::mbar_init(&sm.commit_done, 8);  // the feature-map and epilogue warps, done reading phi
     sm.abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -185,6 +265,22 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
+  // phi and dZ of unit k's block by the eight feature-map and epilogue warps (gt = 0..255):
+  // waits for the staged u_k, writes phi into the lent stage, and once every warp's rows are
+  // there sums this thread's column f = gt into Z.
+  auto commit_phi = [&](const Unit& y, int k, int gt) -> bool {
+    if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.u_staged, k & 1, abort_flag, lim))) return false;
+    uint8_t* phib = sm.s[kCommitStage][0];
+    block_phi(reinterpret_cast<const float*>(sm.s[kCommitStage][1]), phib, gt, y.n);
+    tc::fence_proxy_async_smem();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) tc::mbar_arrive(&sm.phi_ready);
+    if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.phi_ready, k & 1, abort_flag, lim))) return false;
+    atomicAdd(pc.Zw + ((size_t)y.slot * p.Hkv + y.g) * kF + gt, block_dz(phib, gt, y.n));
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) tc::mbar_arrive(&sm.commit_done);  // done reading the lent stage
+    return true;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -559,96 +655,31 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.fin_full[fb]);
 
-      // ---- the commit of this unit: phi of its block rows from u_k = K W_g, whose 32 rows sit
-      // in lane quarter 0 (one thread per row); e+ in place over u_k and e- in the e- columns,
-      // then normalised and rounded to bf16 into the lent stage as the B operand of dS^T:
-      // F quarter a = f / 64, row t, 16-byte chunk (f % 64) / 8 stored at chunk ^ (t % 8)
+      // ---- the commit of this unit: u_k = K W_g, whose 32 block rows sit in lanes 0-7 of the
+      // four TMEM lane quarters (rows 8 wq + lane), is staged in the lent stage's second half
+      // as U [32 rows][128] fp32; then the eight feature-map and epilogue warps form phi and dZ
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.uk_done, k & 1, abort_flag, lim))) break;
       tc::tc_fence_after();
-      uint8_t* phib = sm.s[kCommitStage][0];
       {
-        // lanes 0-7 of each quarter hold block rows 8 wq + lane; the other lanes skip the math
+        float* U = reinterpret_cast<float*>(sm.s[kCommitStage][1]);
         const int t = 8 * wq + (lane & 7);
-        const bool mine = lane < 8;
-        float cmx = -INFINITY, cmn = INFINITY;
 #pragma unroll 1
         for (int c = 0; c < kGroups; ++c) {
           float uu[32];
           tc::tmem_ld32(tl + kColU + c * 32, uu);
           tc::tmem_wait_ld();
+          if (lane < 8) {
+            float4* dst = reinterpret_cast<float4*>(U + t * kFh + c * 32);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            cmx = fmaxf(cmx, uu[i]);
-            cmn = fminf(cmn, uu[i]);
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(uu[4 * i], uu[4 * i + 1], uu[4 * i + 2], uu[4 * i + 3]);
           }
         }
-        const float cbx = cmx * log2e, cbn = cmn * log2e;
-        float csp = 0.f, csm = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < kGroups; ++c) {
-          float uu[32], e2[32];
-          tc::tmem_ld32(tl + kColU + c * 32, uu);
-          tc::tmem_wait_ld();
-          if (mine) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float a = uu[i] * log2e;
-              uu[i] = tc::ex2(a - cbx);
-              e2[i] = tc::ex2(cbn - a);
-              csp += uu[i];
-              csm += e2[i];
-            }
-          }
-          tc::tmem_st32(tl + kColU + c * 32, uu);
-          tc::tmem_st32(tl + kColEm + c * 32, e2);
-        }
-        tc::tmem_wait_st();
-        const bool live = mine && t < x.n;  // rows past the block add nothing
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          const float sc = live ? 1.f / (h ? csm : csp) : 0.f;
-#pragma unroll 1
-          for (int c = 0; c < kGroups; ++c) {
-            float ee[32];
-            tc::tmem_ld32(tl + (h ? kColEm : kColU) + c * 32, ee);
-            tc::tmem_wait_ld();
-            if (mine) {
-              uint8_t* rowp = phib + (2 * h + (c >> 1)) * (kPhiBytes / 4) + t * 128;
-#pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
-                const int ch = 4 * (c & 1) + q4;
-                *reinterpret_cast<uint4*>(rowp + ((ch ^ (t & 7)) << 4)) =
-                    make_uint4(pack_bf16(ee[8 * q4] * sc, ee[8 * q4 + 1] * sc),
-                               pack_bf16(ee[8 * q4 + 2] * sc, ee[8 * q4 + 3] * sc),
-                               pack_bf16(ee[8 * q4 + 4] * sc, ee[8 * q4 + 5] * sc),
-                               pack_bf16(ee[8 * q4 + 6] * sc, ee[8 * q4 + 7] * sc));
-              }
-            }
-          }
-        }
-        tc::fence_proxy_async_smem();
+        // u_k has been read from TMEM (the next unit's u may overwrite it once phi is ready)
         tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&sm.phi_ready);  // this warp's 8 rows of phi are written
+        if (lane == 0) tc::mbar_arrive(&sm.u_staged);
       }
-      // dZ: column sums of the bf16 phi over the block rows (features tid and tid + 128)
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.phi_ready, k & 1, abort_flag, lim))) break;
-      {
-        const int tid = wq * 32 + lane;
-        float* Zg = pc.Zw + ((size_t)x.slot * p.Hkv + x.g) * kF;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int f = tid + hh * kFh, quarter = f >> 6, ch = (f & 63) >> 3, w8 = f & 7;
-          const uint8_t* base = phib + quarter * (kPhiBytes / 4);
-          float acc = 0.f;
-          for (int tt = 0; tt < x.n; ++tt)
-            acc += __bfloat162float(
-                *reinterpret_cast<const __nv_bfloat16*>(base + tt * 128 + ((ch ^ (tt & 7)) << 4) + w8 * 2));
-          atomicAdd(Zg + f, acc);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(&sm.commit_done);  // done reading the lent stage
+      if (!commit_phi(x, k, wq * 32 + lane)) break;
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -696,6 +727,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
         }
       }
 
+      // ---- phi and dZ of this unit's block, with the feature-map warps
+      if (!commit_phi(x, k, (warp - 2) * 32 + lane)) break;
       // ---- the commit of this unit: S[f][d] += dS^T[d][f] by reducing atomic adds straight
       // from the accumulator (lane = d, so each warp instruction adds one 128-byte row piece)
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.ds_full, k & 1, abort_flag, lim))) break;
