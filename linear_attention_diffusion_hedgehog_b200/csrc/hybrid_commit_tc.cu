@@ -11,12 +11,13 @@
 // Each (request, KV head) unit runs the decode step exactly as the decode-only kernel does
 // (the same roles, rings, feature map and shared-normaliser merge; the states are read once,
 // through the S ring), then its commit:
-//   u_k  = K W_g                  bf16 MMA, M 128 (the 32 block rows, loaded again into the
-//                                  ring stage the unit's last state group has released; the
-//                                  other rows are ignored), N 128, into the feature-map
-//                                  columns the unit has finished with
-//   phi  = [softmax(u_k), softmax(-u_k)] per block row: the feature-map warps stage u_k's 32
-//          rows in the stage's second half (fp32), then all eight feature-map and epilogue
+//   u_k  = K W_g                  bf16 MMA, M 128 (the 32 block rows from the unit's own K
+//                                  buffer, which the next unit's K waits for; the other
+//                                  rows are ignored), N 128, into the feature-map columns
+//                                  the unit has finished with
+//   phi  = [softmax(u_k), softmax(-u_k)] per block row: the feature-map warp of TMEM lane
+//          quarter 0 stages u_k's 32 rows in the second half of the ring stage the unit's last
+//          state group has released (fp32), then all eight feature-map and epilogue
 //          warps (idle between the unit's output and its dS^T) form phi, eight threads per row
 //          agreeing on its max, min and sums by shuffles, rounded to bf16 into the stage's
 //          first half (the producer holds the stage back until dS^T and dZ have read it);
@@ -88,11 +89,11 @@ struct __align__(1024) Smem {
   uint8_t p[kPBytes];           // P: [128 rows][64 B], 64-byte swizzle
   float z[2][kF];
   float fin[2][2][kM];          // per unit (double-buffered): epilogue factors c+/den, c-/den
-  uint64_t qk_full, qk_empty, v_full, v_empty, v_ready, z_full[2], z_empty[2];
+  uint64_t q_full, k_full, qk_empty, v_full, v_empty, v_ready, z_full[2], z_empty[2];
   uint64_t s_full[kStages], s_empty[kStages];
   uint64_t e_ready[kGroups], p_ready;
   uint64_t w_full, u_full, acc_full, acc_empty, drain, fin_full[2], fin_empty[2];
-  uint64_t pv_done, kc_full, uk_done, u_staged, phi_ready, ds_full, ds_empty, commit_done;
+  uint64_t uk_done, u_staged, phi_ready, ds_full, ds_empty, commit_done;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -216,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
   const int units = p.R * p.Hkv;
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(&sm.qk_full, 1);
+    tc::mbar_init(&sm.q_full, 1);
+    tc::mbar_init(&sm.k_full, 1);
     tc::mbar_init(&sm.qk_empty, 1);
     tc::mbar_init(&sm.v_full, 1);
     tc::mbar_init(&sm.v_empty, 1);
@@ -238,10 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
     tc::mbar_init(&sm.acc_full, 1);
     tc::mbar_init(&sm.acc_empty, 4);  // the four epilogue warps
     tc::mbar_init(&sm.drain, 1);
-    tc::mbar_init(&sm.pv_done, 1);
-    tc::mbar_init(&sm.kc_full, 1);
     tc::mbar_init(&sm.uk_done, 1);
-    tc::mbar_init(&sm.u_staged, 4);     // the four feature-map warps, 8 block rows each
+    tc::mbar_init(&sm.u_staged, 1);     // the feature-map warp of lane quarter 0 (the block rows)
     tc::mbar_init(&sm.phi_ready, 8);    // the feature-map and epilogue warps, 4 block rows each
     tc::mbar_init(&sm.ds_full, 1);
     tc::mbar_init(&sm.ds_empty, 4);     // the four epilogue warps
@@ -255,7 +255,6 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
     tc::prefetch_tensormap(&p.tm_v);
     tc::prefetch_tensormap(&p.tm_w);
     tc::prefetch_tensormap(&p.tm_s);
-    tc::prefetch_tensormap(&pc.tm_k8);
   }
   if (warp == 1) {
     tc::tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -287,27 +286,12 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
     if (lane == 0) {
       int g_res = -1, q = 0;
       uint32_t w_loads = 0;
-      int armed_qk = -1, armed_v = -1, armed_w = -1, armed_z[2] = {-1, -1}, armed_kc = -1;
-      Unit xp{};  // the previous unit: its K is loaded again for its commit
-      // K of unit j into the lent ring stage, laid out like Q (two d halves 16 KiB apart), block
-      // rows 8 jq .. 8 jq + 7 at tile rows 32 jq .. (so each TMEM lane quarter of u_k holds 8 of
-      // them), once unit j's contraction and P V are done with the stage
-      auto load_kc = [&](const Unit& y, int j) -> bool {
-        if (!tc::mbar_wait(&sm.pv_done, j & 1, abort_flag, lim)) return false;
-        tc::mbar_arrive_expect_tx(&sm.kc_full, kKBytes);
-#pragma unroll
-        for (int jq = 0; jq < 4; ++jq) {
-          tc::tma_load_3d(sm.s[kCommitStage][0] + jq * 4096, &pc.tm_k8, &sm.kc_full, 0, y.g, y.lo + 8 * jq);
-          tc::tma_load_3d(sm.s[kCommitStage][1] + jq * 4096, &pc.tm_k8, &sm.kc_full, 64, y.g, y.lo + 8 * jq);
-        }
-        armed_kc = j & 1;
-        return true;
-      };
+      int armed_q = -1, armed_k = -1, armed_v = -1, armed_w = -1, armed_z[2] = {-1, -1};
       int armed_s[kStages];
 #pragma unroll
       for (int i = 0; i < kStages; ++i) armed_s[i] = -1;
       bool ok = true;
-      int ucur = blockIdx.x, last_k = -1;
+      int ucur = blockIdx.x;
       Unit x{};
       for (int k = 0; ok && next_unit(p, units, &ucur, true, &x); ++k) {
         if (x.g != g_res) {
@@ -322,12 +306,18 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
         }
         if (k >= 1 && !tc::mbar_wait(&sm.qk_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
         // Q: two d halves of 32 G rows, each at the start of its 16 KiB half of the tile
-        tc::mbar_arrive_expect_tx(&sm.qk_full, (kQBytes / kG) * p.G + kKBytes);
-        tc::tma_load_3d(sm.q, &p.tm_q, &sm.qk_full, 0, p.G * x.g, x.lo);
-        tc::tma_load_3d(sm.q + kQBytes / 2, &p.tm_q, &sm.qk_full, 64, p.G * x.g, x.lo);
-        tc::tma_load_3d(sm.k, &p.tm_k, &sm.qk_full, 0, x.g, x.lo);
-        tc::tma_load_3d(sm.k + kKBytes / 2, &p.tm_k, &sm.qk_full, 64, x.g, x.lo);
-        armed_qk = k & 1;
+        tc::mbar_arrive_expect_tx(&sm.q_full, (kQBytes / kG) * p.G);
+        tc::tma_load_3d(sm.q, &p.tm_q, &sm.q_full, 0, p.G * x.g, x.lo);
+        tc::tma_load_3d(sm.q + kQBytes / 2, &p.tm_q, &sm.q_full, 64, p.G * x.g, x.lo);
+        armed_q = k & 1;
+        // K stays until the previous unit's commit has read its own K (u_k): the first unit's
+        // goes out now, the others just ahead of the last S pair (below)
+        if (k == 0) {
+          tc::mbar_arrive_expect_tx(&sm.k_full, kKBytes);
+          tc::tma_load_3d(sm.k, &p.tm_k, &sm.k_full, 0, x.g, x.lo);
+          tc::tma_load_3d(sm.k + kKBytes / 2, &p.tm_k, &sm.k_full, 64, x.g, x.lo);
+          armed_k = 0;
+        }
         const int zb = k & 1, zj = k >> 1;
         if (zj >= 1 && !tc::mbar_wait(&sm.z_empty[zb], (zj - 1) & 1, abort_flag, lim)) { ok = false; break; }
         tc::mbar_arrive_expect_tx(&sm.z_full[zb], kZBytes);
@@ -337,10 +327,16 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
         for (int i = 0; i < kGroups; ++i, ++q) {
           const int grp = group_at(i);
           if (i == kStages - 1) {
-            // the previous unit's commit: its K (once its P V is done), then V of this unit
-            // (once the previous commit's dS^T has read V), then the last S pair goes into the
-            // stage the previous commit borrowed, once that commit is done
-            if (k >= 1 && !load_kc(xp, k - 1)) { ok = false; break; }
+            // this unit's K once the previous unit's commit has read its own (u_k), then V of
+            // this unit (once the previous commit's dS^T has read V), then the last S pair goes
+            // into the stage the previous commit borrowed, once that commit is done
+            if (k >= 1) {
+              if (!tc::mbar_wait(&sm.uk_done, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
+              tc::mbar_arrive_expect_tx(&sm.k_full, kKBytes);
+              tc::tma_load_3d(sm.k, &p.tm_k, &sm.k_full, 0, x.g, x.lo);
+              tc::tma_load_3d(sm.k + kKBytes / 2, &p.tm_k, &sm.k_full, 64, x.g, x.lo);
+              armed_k = k & 1;
+            }
             if (k >= 1 && !tc::mbar_wait(&sm.v_empty, (k - 1) & 1, abort_flag, lim)) { ok = false; break; }
             tc::mbar_arrive_expect_tx(&sm.v_full, kKBytes);
             tc::tma_load_3d(sm.v, &p.tm_v, &sm.v_full, 0, x.g, x.lo);
@@ -359,21 +355,17 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
                               srow0 + hf * kFh + grp * kChunk);
           armed_s[st] = j & 1;
         }
-        xp = x;
-        last_k = k;
       }
-      // the last unit's commit needs its K too
-      if (ok && last_k >= 0) load_kc(xp, last_k);
       // Drain: every copy this thread started has landed before the CTA can exit.
       volatile int never = 0;
-      if (armed_qk >= 0) tc::mbar_wait(&sm.qk_full, armed_qk, &never, lim);
+      if (armed_q >= 0) tc::mbar_wait(&sm.q_full, armed_q, &never, lim);
+      if (armed_k >= 0) tc::mbar_wait(&sm.k_full, armed_k, &never, lim);
       if (armed_v >= 0) tc::mbar_wait(&sm.v_full, armed_v, &never, lim);
       for (int b = 0; b < 2; ++b)
         if (armed_z[b] >= 0) tc::mbar_wait(&sm.z_full[b], armed_z[b], &never, lim);
       for (int c = 0; c < kStages; ++c)
         if (armed_s[c] >= 0) tc::mbar_wait(&sm.s_full[c], armed_s[c], &never, lim);
       if (armed_w >= 0) tc::mbar_wait(&sm.w_full, armed_w, &never, lim);
-      if (armed_kc >= 0) tc::mbar_wait(&sm.kc_full, armed_kc, &never, lim);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -391,7 +383,6 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
       const uint32_t wa = tc::smem_u32(sm.w);
       const uint32_t qa = tc::smem_u32(sm.q);
       const uint32_t ka = tc::smem_u32(sm.k);
-      const uint32_t kca = tc::smem_u32(sm.s[kCommitStage][0]);     // K again, for u_k
       const uint32_t phia = tc::smem_u32(sm.s[kCommitStage][0]);    // phi of the block
       // u = Q W_g and s = Q K^T of unit j
       auto issue_uqk = [&](const Unit& y, int j) -> bool {
@@ -400,7 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
           ++w_seen;
           g_res = y.g;
         }
-        if (!tc::mbar_wait(&sm.qk_full, j & 1, abort_flag, lim)) return false;
+        if (!tc::mbar_wait(&sm.q_full, j & 1, abort_flag, lim)) return false;
+        if (!tc::mbar_wait(&sm.k_full, j & 1, abort_flag, lim)) return false;
         tc::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
@@ -459,13 +451,14 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
           tc::mma_bf16_ss(tbase + kColAp, a, b, kIdPV, 1);
         }
         tc::mma_commit(&sm.acc_full);
-        tc::mma_commit(&sm.pv_done);
         // commit: u_k = K W_g (the block's 32 rows lead the 128-row tile) into u's columns
-        if (!tc::mbar_wait(&sm.kc_full, k & 1, abort_flag, lim)) { ok = false; break; }
+        // u_k reads K from its own buffer, still holding this unit's K: an M = 128 tile whose
+        // rows 32 .. 127 run on into the V and P buffers (in bounds, and not written until
+        // this unit's dS^T and the next unit's P); those rows of u_k are never read
         tc::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint64_t a = tc::smem_desc(kca + (kk >> 2) * kSBytes + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
+          const uint64_t a = tc::smem_desc(ka + (kk >> 2) * (kKBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
           const uint64_t b = tc::smem_desc(wa + kk * 2048, kWBytes / 2, 1024, tc::kSwizzle128B);
           tc::mma_bf16_ss(tbase + kColU, a, b, kIdQW, kk > 0);
         }
@@ -655,24 +648,21 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.fin_full[fb]);
 
-      // ---- the commit of this unit: u_k = K W_g, whose 32 block rows sit in lanes 0-7 of the
-      // four TMEM lane quarters (rows 8 wq + lane), is staged in the lent stage's second half
-      // as U [32 rows][128] fp32; then the eight feature-map and epilogue warps form phi and dZ
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.uk_done, k & 1, abort_flag, lim))) break;
-      tc::tc_fence_after();
-      {
+      // ---- the commit of this unit: u_k = K W_g, whose 32 block rows sit in TMEM lanes 0-31
+      // (lane quarter 0), is staged by that quarter's warp in the lent stage's second half as
+      // U [32 rows][128] fp32; then the eight feature-map and epilogue warps form phi and dZ
+      if (wq == 0) {
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.uk_done, k & 1, abort_flag, lim))) break;
+        tc::tc_fence_after();
         float* U = reinterpret_cast<float*>(sm.s[kCommitStage][1]);
-        const int t = 8 * wq + (lane & 7);
 #pragma unroll 1
         for (int c = 0; c < kGroups; ++c) {
           float uu[32];
           tc::tmem_ld32(tl + kColU + c * 32, uu);
           tc::tmem_wait_ld();
-          if (lane < 8) {
-            float4* dst = reinterpret_cast<float4*>(U + t * kFh + c * 32);
+          float4* dst = reinterpret_cast<float4*>(U + lane * kFh + c * 32);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_float4(uu[4 * i], uu[4 * i + 1], uu[4 * i + 2], uu[4 * i + 3]);
-          }
+          for (int i = 0; i < 8; ++i) dst[i] = make_float4(uu[4 * i], uu[4 * i + 1], uu[4 * i + 2], uu[4 * i + 3]);
         }
         // u_k has been read from TMEM (the next unit's u may overwrite it once phi is ready)
         tc::tc_fence_before();
@@ -792,13 +782,6 @@ cudaError_t launch_hybrid_commit_tc(const HybridArgs& a, float* S, float* Z, cud
     const uint64_t strides[1] = {kD * 4};
     const uint32_t box[2] = {32, kChunk};
     if (!make_tensor_map(&p.tm_s, true, 2, a.S, dims, strides, box, kTma128BAtom32)) return cudaErrorInvalidValue;
-  }
-  {
-    // K again for the commit, 8 block rows per box
-    const uint64_t dims[3] = {kD, (uint64_t)a.Hkv, T};
-    const uint64_t strides[2] = {kD * 2, (uint64_t)a.Hkv * kD * 2};
-    const uint32_t box[3] = {64, 1, 8};
-    if (!make_tensor_map(&pc.tm_k8, false, 3, a.K, dims, strides, box, kTma128B)) return cudaErrorInvalidValue;
   }
   pc.Sw = S;
   pc.Zw = Z;

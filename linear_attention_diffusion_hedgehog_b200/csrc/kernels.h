@@ -67,7 +67,6 @@ struct TcHybridParams {
 // step's, plus K in 8-row boxes for the commit, and S and Z for its atomic adds.
 struct TcHybridCommitParams {
   TcHybridParams h;
-  CUtensorMap tm_k8;
   float* Sw;
   float* Zw;
 };
