@@ -31,8 +31,9 @@
 //                                  128-byte row piece); the lines were read by this unit's
 //                                  state stream moments before, so L2 serves the
 //                                  read-modify-write and S crosses HBM once each way.
-// The next unit's u and s are issued once phi is in shared memory, so its feature map runs
-// while dS^T is formed and drained.
+// dS^T is issued as soon as phi is in shared memory and the output has been read, and the
+// next unit's u and s right after it, so the drain starts early and the next unit's feature
+// map runs while dS^T is drained.
 //
 // Every wait is bounded; on expiry the CTA raises BHA_ERR_TIMEOUT in dev_err, drains its
 // own copies and MMAs, frees its TMEM and returns.
@@ -132,20 +133,21 @@ __device__ __forceinline__ bool next_unit(const TcHybridParams& p, int units, in
   return false;
 }
 
-// phi of the block's rows from u_k staged in shared memory (U: [32 rows][128] fp32), by the
-// eight feature-map and epilogue warps: thread gt (0..255) owns row gt / 8 and u columns
-// 16 (gt % 8) .. + 15, so the eight lanes of a row agree on its max, min and sums by
-// shuffles.  phi = [e+ / sum e+, e- / sum e-] rounded to bf16 into phib as the B operand of
-// dS^T: F quarter a = f / 64, row t, 16-byte chunk (f % 64) / 8 stored at chunk ^ (t % 8);
-// rows past the block (t >= n) are written as zeros.
+// phi of the block's rows from u_k staged in shared memory (U: [32 rows][128] fp32, float4
+// slot j of row t at slot j ^ (t % 8)), by the eight feature-map and epilogue warps: thread
+// gt (0..255) owns row t = gt / 8 and the float4 slots s8 + 8 i (i = 0..3, s8 = gt % 8), i.e.
+// u columns 4 s8 + 32 i + m, so the eight lanes of a row read eight different bank groups and
+// agree on its max, min and sums by shuffles.  phi = [e+ / sum e+, e- / sum e-] rounded to
+// bf16 into phib as the B operand of dS^T: F quarter a = f / 64, row t, 16-byte chunk
+// (f % 64) / 8 stored at chunk ^ (t % 8); rows past the block (t >= n) are written as zeros.
 __device__ __forceinline__ void block_phi(const float* U, uint8_t* phib, int gt, int n) {
   const float log2e = 1.4426950408889634f;
   const int t = gt >> 3, s8 = gt & 7;
   float u[16];
-  const float4* src = reinterpret_cast<const float4*>(U + t * kFh + 16 * s8);
+  const float4* src = reinterpret_cast<const float4*>(U + t * kFh);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float4 v = src[i];
+    const float4 v = src[(s8 + 8 * i) ^ (t & 7)];
     u[4 * i] = v.x;
     u[4 * i + 1] = v.y;
     u[4 * i + 2] = v.z;
@@ -183,16 +185,15 @@ __device__ __forceinline__ void block_phi(const float* U, uint8_t* phib, int gt,
   for (int h = 0; h < 2; ++h) {
     const float* e = h ? em : ep;
     const float sc = h ? im : ip;
-    // features h F/2 + 16 s8 + i: F quarter 2 h + s8 / 4, chunks 2 (s8 % 4) and 2 (s8 % 4) + 1
-    uint8_t* rowp = phib + (2 * h + (s8 >> 2)) * (kPhiBytes / 4) + t * 128;
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int ch = 2 * (s8 & 3) + q;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (live)
-        v = make_uint4(pack_bf16(e[8 * q] * sc, e[8 * q + 1] * sc), pack_bf16(e[8 * q + 2] * sc, e[8 * q + 3] * sc),
-                       pack_bf16(e[8 * q + 4] * sc, e[8 * q + 5] * sc), pack_bf16(e[8 * q + 6] * sc, e[8 * q + 7] * sc));
-      *reinterpret_cast<uint4*>(rowp + ((ch ^ (t & 7)) << 4)) = v;
+    for (int i = 0; i < 4; ++i) {
+      // features h F/2 + 4 s8 + 32 i + (0..3): F quarter 2 h + i / 2, chunk s8 / 2 + 4 (i % 2),
+      // bytes 8 (s8 % 2) .. + 7 of the chunk
+      const int ch = (s8 >> 1) + 4 * (i & 1);
+      uint8_t* dst = phib + (2 * h + (i >> 1)) * (kPhiBytes / 4) + t * 128 + ((ch ^ (t & 7)) << 4) + (s8 & 1) * 8;
+      uint2 v = make_uint2(0, 0);
+      if (live) v = make_uint2(pack_bf16(e[4 * i] * sc, e[4 * i + 1] * sc), pack_bf16(e[4 * i + 2] * sc, e[4 * i + 3] * sc));
+      *reinterpret_cast<uint2*>(dst) = v;
     }
   }
 }
@@ -463,11 +464,10 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
           tc::mma_bf16_ss(tbase + kColU, a, b, kIdQW, kk > 0);
         }
         tc::mma_commit(&sm.uk_done);
-        // phi in shared memory: u_k has been read, so the next unit's u and s may follow
+        // dS^T = V^T phi over the accumulator columns, once phi is in shared memory and the
+        // epilogue has read the output (first, so that its drain, which the next unit's
+        // contraction waits for, starts as early as possible)
         if (!tc::mbar_wait(&sm.phi_ready, k & 1, abort_flag, lim)) { ok = false; break; }
-        const bool have_next = next_unit(p, units, &ucur, false, &xn);
-        if (have_next && !issue_uqk(xn, k + 1)) { ok = false; break; }
-        // dS^T = V^T phi over the accumulator columns once the epilogue has read the output
         if (!tc::mbar_wait(&sm.acc_empty, k & 1, abort_flag, lim)) { ok = false; break; }
         tc::tc_fence_after();
 #pragma unroll
@@ -480,6 +480,9 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
         }
         tc::mma_commit(&sm.ds_full);
         tc::mma_commit(&sm.v_empty);
+        // then the next unit's u and s (u_k, in u's columns, was staged before phi was ready)
+        const bool have_next = next_unit(p, units, &ucur, false, &xn);
+        if (have_next && !issue_uqk(xn, k + 1)) { ok = false; break; }
         x = xn;
         have = have_next;
       }
@@ -660,9 +663,12 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
           float uu[32];
           tc::tmem_ld32(tl + kColU + c * 32, uu);
           tc::tmem_wait_ld();
-          float4* dst = reinterpret_cast<float4*>(U + lane * kFh + c * 32);
+          // float4 slot j of row `lane` at slot j ^ (lane % 8): the eight lanes of each
+          // quarter-warp store into eight different bank groups
+          float4* dst = reinterpret_cast<float4*>(U + lane * kFh);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) dst[i] = make_float4(uu[4 * i], uu[4 * i + 1], uu[4 * i + 2], uu[4 * i + 3]);
+          for (int i = 0; i < 8; ++i)
+            dst[(c * 8 + i) ^ (lane & 7)] = make_float4(uu[4 * i], uu[4 * i + 1], uu[4 * i + 2], uu[4 * i + 3]);
         }
         // u_k has been read from TMEM (the next unit's u may overwrite it once phi is ready)
         tc::tc_fence_before();
