@@ -220,6 +220,12 @@ __device__ __forceinline__ float phi_column_sum(const uint8_t* base, int n, int 
   return sum;
 }
 
+// The four-sum form as a call of its own, so that its registers are allocated apart from the
+// feature map's (inlined, it pushes the 64- and 128-row instantiations into spills).
+__device__ __noinline__ float phi_column_sum4(const uint8_t* base, int n, int ch) {
+  return phi_column_sum<4>(base, n, ch);
+}
+
 template <int kBt>
 __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_constant__ TcCommitParams p) {
   constexpr int kReq = Shape<kBt>::kReq;
@@ -452,17 +458,19 @@ __global__ void __launch_bounds__(kThreads, 1) commit_tc_kernel(const __grid_con
       // have written theirs, the dS^T products may start
       tc::fence_proxy_async_smem();
       // ---- dZ[j][f] = sum over the block's tokens of the bf16 phi (thread tid owns f = tid).
-      // With four requests per tile it is summed before phi is handed to the dS^T products
-      // (one running sum: the register budget has no room for more); with one or two it is
-      // summed while the first product runs, four partial sums at a time.  (Both measured:
-      // 30.9 us and 41.7 us at 32- and 128-token blocks, against 31.8 and 52.1 us the other
-      // way round.)
+      // With four requests per tile it is summed before phi is handed to the dS^T products,
+      // one running sum; with one or two it is summed while the first product runs, four
+      // partial sums at a time in a call of its own.  Measured at 32- and 128-token blocks:
+      // 30.9-31.2 us and 39.7 us this way; 31.8 us with the four-sum call before the hand-off
+      // at 32 tokens, 52.1 us with the one-sum form before the hand-off at 128.
       const int zf = tid, zq = zf >> 6, zch = (zf & 63) >> 3, zw = zf & 7;
       auto column_sums = [&](auto acc_tag) {
         constexpr int kAcc = decltype(acc_tag)::value;
 #pragma unroll 1
-        for (int j = 0; j < kReq; ++j)
-          sm.dz[j][zf] = phi_column_sum<kAcc>(sm.phi[j] + zq * (kPhiReqBytes / 4) + zw * 2, rq[j].n, zch);
+        for (int j = 0; j < kReq; ++j) {
+          const uint8_t* base = sm.phi[j] + zq * (kPhiReqBytes / 4) + zw * 2;
+          sm.dz[j][zf] = kAcc == 1 ? phi_column_sum<1>(base, rq[j].n, zch) : phi_column_sum4(base, rq[j].n, zch);
+        }
       };
       if constexpr (kBt == 32) {
         tc::tc_fence_before();
