@@ -16,12 +16,13 @@
 //   warp 1      TMEM owner and MMA issuer: u of tile k into TMEM buffer k % 2 (two buffers of
 //               256 columns: u, overwritten in place by e+, then e-), so the next tile's MMA
 //               overlaps this tile's epilogue.
-//   warps 2-9   two warps per TMEM lane quarter: warps 2-5 take u columns 0-63, warps 6-9
-//               columns 64-127 of their 32 rows.  Each computes max / min and the partial sums
-//               of its columns, exchanges them with its partner through shared memory, writes
-//               e+ and e- to TMEM, then reads them back normalised, 32 rows x 128 bytes at a
-//               time, into a double-buffered staging slot that one asynchronous bulk tensor
-//               store writes to phi.
+//   warps 2-9   two groups of four, taking alternate tiles (warps 2-5 the even ones, 6-9 the
+//               odd ones, matching the TMEM buffers), so one group's exponentials overlap the
+//               other group's read-out and stores.  In a group, warp wq owns TMEM lane quarter
+//               wq and each thread one whole row: max and min of its 128 u values, e+ and e-
+//               written to TMEM with their sums, then read back normalised, 32 rows x 128
+//               bytes at a time, into a double-buffered staging slot that one asynchronous
+//               bulk tensor store writes to phi.
 //
 // Every wait is bounded.  On expiry the CTA stops early and this call's output is undefined
 // (the feature-map entry point has no error word); nothing traps and TMEM is freed.
@@ -50,7 +51,6 @@ struct __align__(1024) Smem {
   uint8_t x[2][kXBytes];
   uint8_t w[kWBytes];
   uint8_t stg[8][2][kStgBytes];  // per epilogue warp, two staging slots (128-byte swizzle)
-  float xch[4][2][kM];           // per-row values the two warps of a lane quarter exchange
   uint64_t x_full[2], x_empty[2], u_full[2], tm_empty[2], w_full, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kThreads, 1) featuremap_tc_kernel(const __grid
       tc::mbar_init(&sm.x_full[i], 1);
       tc::mbar_init(&sm.x_empty[i], 1);
       tc::mbar_init(&sm.u_full[i], 1);
-      tc::mbar_init(&sm.tm_empty[i], 8);
+      tc::mbar_init(&sm.tm_empty[i], 4);  // the four warps of the tile's group
     }
     tc::mbar_init(&sm.w_full, 1);
     tc::mbar_init(&sm.drain, 1);
@@ -166,48 +166,48 @@ __global__ void __launch_bounds__(kThreads, 1) featuremap_tc_kernel(const __grid
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
+    // Two groups of four warps take alternate tiles (warps 2-5 the even ones, 6-9 the odd
+    // ones, matching the two TMEM buffers), so one group's exponentials (MUFU) overlap the
+    // other group's read-out and stores.  In a group, warp wq owns TMEM lane quarter wq and
+    // each thread one whole row.
     const int sw = warp - 2;         // 0..7
-    const int part = sw >> 2;        // 0: u columns 0-63, 1: columns 64-127
+    const int grp = sw >> 2;         // tile parity this warp's group takes
     const int wq = warp & 3;         // TMEM lane quarter this warp may access
-    const int row = wq * 32 + lane;  // tile row
     const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
-    const uint32_t pair_bar = 2 + wq;
     const float log2e = 1.4426950408889634f;
-    float* mine = &sm.xch[0][part][row];
-    const float* theirs = &sm.xch[0][part ^ 1][row];
-    constexpr int kX = 2 * kM;       // stride between exchange slots
     const int row0 = wq * 32;  // the warp's 32 rows are one store box (see the host side)
     bool good = true;
-    int k = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++k) {
-      const int g = t % p.Hw, t0 = (t / p.Hw) * tok_per_tile, b = k & 1;
+    int k = 0, nst = 0;  // nst: bulk stores this warp has committed (staging slot rotation)
+    for (int t = blockIdx.x; good && t < tiles; t += gridDim.x, ++k) {
+      const int b = k & 1;
+      if (b != grp) continue;
+      const int g = t % p.Hw, t0 = (t / p.Hw) * tok_per_tile;
       const uint32_t tb = tl + b * 256;
-      good = tc::mbar_wait(&sm.u_full[b], (k >> 1) & 1, abort_flag, lim) && good;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.u_full[b], (k >> 1) & 1, abort_flag, lim))) { good = false; break; }
       tc::tc_fence_after();
 
-      float u0[32], u1[32];
-      tc::tmem_ld32(tb + part * 64, u0);
-      tc::tmem_ld32(tb + part * 64 + 32, u1);
-      tc::tmem_wait_ld();
+      // max and min of the row's 128 u values
       float mx = -INFINITY, mn = INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < kFh / 32; c += 2) {
+        float u0[32], u1[32];
+        tc::tmem_ld32(tb + c * 32, u0);
+        tc::tmem_ld32(tb + c * 32 + 32, u1);
+        tc::tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        mx = fmaxf(mx, fmaxf(u0[i], u1[i]));
-        mn = fminf(mn, fminf(u0[i], u1[i]));
+        for (int i = 0; i < 32; ++i) {
+          mx = fmaxf(mx, fmaxf(u0[i], u1[i]));
+          mn = fminf(mn, fminf(u0[i], u1[i]));
+        }
       }
-      mine[0 * kX] = mx;
-      mine[1 * kX] = mn;
-      tc::named_barrier_sync(pair_bar, 64);
-      mx = fmaxf(mx, theirs[0 * kX]);
-      mn = fminf(mn, theirs[1 * kX]);
-
-      // unnormalised e+ over u in place and e- beside it, with their partial sums
+      // unnormalised e+ over u in place and e- beside it, with their sums
       const float bpl = mx * log2e, bml = mn * log2e;
       float esp = 0.f, esm = 0.f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float(&uu)[32] = h ? u1 : u0;
-        float ep[32];
+#pragma unroll 1
+      for (int c = 0; c < kFh / 32; ++c) {
+        float uu[32], ep[32];
+        tc::tmem_ld32(tb + c * 32, uu);
+        tc::tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float a = uu[i] * log2e;
@@ -216,47 +216,43 @@ __global__ void __launch_bounds__(kThreads, 1) featuremap_tc_kernel(const __grid
           esp += ep[i];
           esm += uu[i];
         }
-        tc::tmem_st32(tb + part * 64 + 32 * h, ep);
-        tc::tmem_st32(tb + 128 + part * 64 + 32 * h, uu);
+        tc::tmem_st32(tb + c * 32, ep);
+        tc::tmem_st32(tb + 128 + c * 32, uu);
       }
       tc::tmem_wait_st();
-      mine[2 * kX] = esp;
-      mine[3 * kX] = esm;
-      // the pair also agrees here whether to go on
-      if (tc::named_barrier_any(pair_bar, 64, !good)) break;
-      const float ip = 1.f / (esp + theirs[2 * kX]);
-      const float im = 1.f / (esm + theirs[3 * kX]);
+      const float ip = 1.f / esp, im = 1.f / esm;
 
-      // phi, 32 rows x 128 bytes per store: fp32 in four chunks of 32 columns (e+ then e-),
-      // bf16 in two chunks of 64 columns
+      // phi, 32 rows x 128 bytes per store: fp32 in eight chunks of 32 columns (e+ then e-),
+      // bf16 in four chunks of 64 columns
       const int tok_w = t0 + row0 / p.G;       // first token of this warp's rows
       const int head_w = g * p.G + row0 % p.G;  // first head of this warp's rows
       const bool store = tok_w < p.T;
-      const int nchunks = p.out_bf16 ? 2 : 4;
+      const int nchunks = p.out_bf16 ? 4 : 8;
       for (int c = 0; c < nchunks; ++c) {
-        const int half = p.out_bf16 ? c : (c >> 1);  // 0: e+, 1: e-
-        const float sc = half ? im : ip;
         uint32_t packed[32];
         int f0;  // first phi column of the chunk
         if (p.out_bf16) {
+          const int half = c >> 1, cc = c & 1;  // 64 columns of e+ or e-
+          const float sc = half ? im : ip;
           float a[32], bb[32];
-          tc::tmem_ld32(tb + half * 128 + part * 64, a);
-          tc::tmem_ld32(tb + half * 128 + part * 64 + 32, bb);
+          tc::tmem_ld32(tb + half * 128 + cc * 64, a);
+          tc::tmem_ld32(tb + half * 128 + cc * 64 + 32, bb);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             packed[i] = pack_bf16(a[2 * i] * sc, a[2 * i + 1] * sc);
             packed[16 + i] = pack_bf16(bb[2 * i] * sc, bb[2 * i + 1] * sc);
           }
-          f0 = half * kFh + part * 64;
+          f0 = half * kFh + cc * 64;
         } else {
-          const int h = c & 1;
+          const int half = c >> 2, cc = c & 3;  // 32 columns of e+ or e-
+          const float sc = half ? im : ip;
           float a[32];
-          tc::tmem_ld32(tb + half * 128 + part * 64 + 32 * h, a);
+          tc::tmem_ld32(tb + half * 128 + cc * 32, a);
           tc::tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) packed[i] = __float_as_uint(a[i] * sc);
-          f0 = half * kFh + part * 64 + 32 * h;
+          f0 = half * kFh + cc * 32;
         }
         if (c == nchunks - 1) {
           // every TMEM read of this tile is done: the MMA may refill the buffer
@@ -264,8 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1) featuremap_tc_kernel(const __grid
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&sm.tm_empty[b]);
         }
-        // staging slot c % 2: its previous store (two chunks ago) must have read it
-        uint8_t* slot = sm.stg[sw][c & 1];
+        // staging slot nst % 2: its previous store (two stores ago) must have read it
+        uint8_t* slot = sm.stg[sw][nst & 1];
         if (lane == 0) bulk_wait_read_one();
         __syncwarp();
 #pragma unroll
@@ -274,9 +270,12 @@ __global__ void __launch_bounds__(kThreads, 1) featuremap_tc_kernel(const __grid
               make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
         tc::fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && store) {
-          tc::tma_store_3d(&p.tm_o, slot, f0, head_w, tok_w);
-          tc::bulk_commit();
+        if (store) {
+          if (lane == 0) {
+            tc::tma_store_3d(&p.tm_o, slot, f0, head_w, tok_w);
+            tc::bulk_commit();
+          }
+          ++nst;
         }
       }
     }
