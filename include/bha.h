@@ -80,9 +80,17 @@ typedef struct {
  * Uses dims->{num_kv_heads, head_dim, feature_dim, total_tokens, act_dtype}.
  * bf16 x with d = 128, F = 256 and x_heads / num_kv_heads a power of two <= 128 (x_heads a
  * multiple of num_kv_heads) takes the tensor-core kernel; its bounded waits have no error word
- * here, so if one ever gave up the output of that call would be undefined (nothing traps). */
+ * here, so if one ever gave up the output of that call would be undefined (nothing traps).
+ * bha_featuremap_checked reports that case. */
 int bha_featuremap(const bha_dims* dims, const void* x, int32_t x_heads, const void* W,
                    void* phi, int32_t out_dtype, void* stream);
+
+/* bha_featuremap with an error word: dev_err is a DEVICE int32 (4-byte aligned) or NULL.  The
+ * tensor-core kernel writes BHA_ERR_TIMEOUT there if one of its bounded waits gave up (the
+ * output of the call is then undefined); nothing is written otherwise, so the caller zeroes it
+ * first.  Host-side validation and return values are those of bha_featuremap.  (ABI 1.01) */
+int bha_featuremap_checked(const bha_dims* dims, const void* x, int32_t x_heads, const void* W,
+                           void* phi, int32_t out_dtype, int32_t* dev_err, void* stream);
 
 /* One denoising step of one block-hybrid layer (§3.1: within-block softmax sums, cross-block
  * read lin_num = phi(q)^T S, lin_den = phi(q)^T Z, and the gated shared-normaliser merge).

@@ -46,6 +46,7 @@ _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
 _SIGS = {
     "bha_featuremap": (ctypes.c_int, [ctypes.POINTER(Dims), _P, _I32, _P, _P, _I32, _P]),
+    "bha_featuremap_checked": (ctypes.c_int, [ctypes.POINTER(Dims), _P, _I32, _P, _P, _I32, _P, _P]),
     "bha_hybrid_attn": (ctypes.c_int, [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                        _P, _P, _P]),
     "bha_commit_block": (ctypes.c_int, [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, _P, _P, _P,
@@ -147,8 +148,10 @@ def kernel_variant(dims: Dims, which: int) -> int:
 
 # ----------------------------------------------------------------------- entry points
 
-def featuremap(x, W, out_dtype=torch.float32, out=None, stream=None):
-    """phi(x) = [softmax(xW), softmax(-xW)] per head.  x [T, H, d]; W [Hkv, d, F/2]."""
+def featuremap(x, W, out_dtype=torch.float32, out=None, dev_err=None, stream=None):
+    """phi(x) = [softmax(xW), softmax(-xW)] per head.  x [T, H, d]; W [Hkv, d, F/2].
+    dev_err: optional device int32 tensor of one element that receives BHA_ERR_TIMEOUT if the
+    kernel's watchdog gave up (bha_featuremap_checked)."""
     _cuda(x, "x", ndim=3)
     _cuda(W, "W", dtype=x.dtype, ndim=3)
     T, H, d = x.shape
@@ -160,8 +163,14 @@ def featuremap(x, W, out_dtype=torch.float32, out=None, stream=None):
     _need(tuple(out.shape) == (T, H, 2 * Fh), "out must be [T, H, F]")
     dims = make_dims(0, Hkv, Hkv, d, 2 * Fh, 1, T, 0, x.dtype)  # R, Hq, slots unused here
     with torch.cuda.device(x.device):  # the library uses the current device
-        st = lib().bha_featuremap(ctypes.byref(dims), _ptr(x), H, _ptr(W), _ptr(out),
-                                  _DTYPE_CODE[out_dtype], _stream(x.device, stream))
+        if dev_err is None:
+            st = lib().bha_featuremap(ctypes.byref(dims), _ptr(x), H, _ptr(W), _ptr(out),
+                                      _DTYPE_CODE[out_dtype], _stream(x.device, stream))
+        else:
+            _cuda(dev_err, "dev_err", dtype=torch.int32)
+            st = lib().bha_featuremap_checked(ctypes.byref(dims), _ptr(x), H, _ptr(W), _ptr(out),
+                                              _DTYPE_CODE[out_dtype], _ptr(dev_err),
+                                              _stream(x.device, stream))
     _check(st, "bha_featuremap")
     return out
 

@@ -8,7 +8,7 @@
 
 namespace {
 
-constexpr int kVersion = 100;
+constexpr int kVersion = 101;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -101,6 +101,11 @@ int bha_kernel_variant(const bha_dims* dims, int32_t which) {
 
 int bha_featuremap(const bha_dims* dims, const void* x, int32_t x_heads, const void* W,
                    void* phi, int32_t out_dtype, void* stream) {
+  return bha_featuremap_checked(dims, x, x_heads, W, phi, out_dtype, nullptr, stream);
+}
+
+int bha_featuremap_checked(const bha_dims* dims, const void* x, int32_t x_heads, const void* W,
+                           void* phi, int32_t out_dtype, int32_t* dev_err, void* stream) {
   int s = check_dims(dims);
   if (s != BHA_OK) return s;
   if (x_heads < 1) return BHA_ERR_INVALID;
@@ -108,10 +113,11 @@ int bha_featuremap(const bha_dims* dims, const void* x, int32_t x_heads, const v
   if (dims->total_tokens == 0) return BHA_OK;
   if (!tensor_ok(x) || !tensor_ok(W) || !tensor_ok(phi)) return BHA_ERR_INVALID;
   if (x == phi || W == phi) return BHA_ERR_INVALID;
+  if (dev_err != nullptr && !index_ok(dev_err)) return BHA_ERR_INVALID;
   if (bha::featuremap_tc_supports(dims->total_tokens, x_heads, dims->num_kv_heads, dims->head_dim,
                                   dims->feature_dim, dims->act_dtype == BHA_BF16))
     return launch_status(bha::launch_featuremap_tc(x, dims->total_tokens, x_heads, dims->num_kv_heads,
-                                                   W, phi, out_dtype == BHA_BF16,
+                                                   W, phi, out_dtype == BHA_BF16, dev_err,
                                                    static_cast<cudaStream_t>(stream)));
   return launch_status(bha::launch_featuremap_simt(
       x, dims->total_tokens, x_heads, dims->num_kv_heads, dims->head_dim, dims->feature_dim, W,

@@ -24,8 +24,8 @@
 //               bytes at a time, into a double-buffered staging slot that one asynchronous
 //               bulk tensor store writes to phi.
 //
-// Every wait is bounded.  On expiry the CTA stops early and this call's output is undefined
-// (the feature-map entry point has no error word); nothing traps and TMEM is freed.
+// Every wait is bounded.  On expiry the CTA stops early, the call's output is undefined and
+// BHA_ERR_TIMEOUT goes to dev_err when the caller passed one; nothing traps and TMEM is freed.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -286,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) featuremap_tc_kernel(const __grid
   __syncthreads();
   tc::tc_fence_after();
   if (warp == 1) tc::tmem_dealloc(tbase, kTmemCols);
+  if (threadIdx.x == 0 && sm.abort_flag) set_error(p.dev_err, BHA_ERR_TIMEOUT);
 }
 
 }  // namespace
@@ -298,7 +299,7 @@ bool featuremap_tc_supports(int T, int x_heads, int Hw, int d, int F, bool act_b
 }
 
 cudaError_t launch_featuremap_tc(const void* x, int T, int x_heads, int Hw, const void* W, void* phi,
-                                 bool out_bf16, cudaStream_t st) {
+                                 bool out_bf16, int32_t* dev_err, cudaStream_t st) {
   TcFeatParams p;
   const int G = x_heads / Hw;
   {
@@ -328,6 +329,7 @@ cudaError_t launch_featuremap_tc(const void* x, int T, int x_heads, int Hw, cons
   p.G = G;
   p.out_bf16 = out_bf16 ? 1 : 0;
   p.wait_limit = 2000000000ll;  // about one second of SM cycles
+  p.dev_err = dev_err;
 
   const int tok_per_tile = kM / G;
   const int tiles = Hw * ((T + tok_per_tile - 1) / tok_per_tile);

@@ -100,6 +100,7 @@ struct TcFullParams {
 // Parameters of the tensor-core feature-map kernel (featuremap_tc.cu).
 struct TcFeatParams {
   CUtensorMap tm_x, tm_w, tm_o;
+  int32_t* dev_err;  // BHA_ERR_TIMEOUT if a bounded wait gave up; may be null
   int T, H, Hw, G, out_bf16;
   long long wait_limit;
 };
@@ -123,7 +124,7 @@ size_t full_prefix_tc_workspace(const FullPrefixArgs& a);
 cudaError_t launch_full_prefix_tc(const FullPrefixArgs& a, void* workspace, cudaStream_t st);
 bool featuremap_tc_supports(int T, int x_heads, int Hw, int d, int F, bool act_bf16);
 cudaError_t launch_featuremap_tc(const void* x, int T, int x_heads, int Hw, const void* W, void* phi,
-                                 bool out_bf16, cudaStream_t st);
+                                 bool out_bf16, int32_t* dev_err, cudaStream_t st);
 
 // generic CUDA-core kernels (simt.cu)
 bool simt_supports(int d, int F, int Bmax);

@@ -105,6 +105,11 @@ def test_featuremap_validation():
     assert L.bha_featuremap(ctypes.byref(dm), MIS, 4, A16b, A16c, 0, NULL) == bha.BHA_ERR_INVALID
     assert L.bha_featuremap(ctypes.byref(dm), A16, 4, A16b, A16, 0, NULL) == bha.BHA_ERR_INVALID
     assert L.bha_featuremap(ctypes.byref(dims(T=0)), A16, 4, A16b, A16c, 0, NULL) == bha.BHA_OK
+    # the checked form validates the same way, plus a misaligned error word
+    assert L.bha_featuremap_checked(ctypes.byref(dm), A16, 0, A16b, A16c, 0, NULL, NULL) == bha.BHA_ERR_INVALID
+    assert L.bha_featuremap_checked(ctypes.byref(dm), MIS, 4, A16b, A16c, 0, NULL, NULL) == bha.BHA_ERR_INVALID
+    assert L.bha_featuremap_checked(ctypes.byref(dm), A16, 4, A16b, A16c, 0, P(0x20001), NULL) == bha.BHA_ERR_INVALID
+    assert L.bha_featuremap_checked(ctypes.byref(dims(T=0)), A16, 4, A16b, A16c, 0, P(0x20000), NULL) == bha.BHA_OK
 
 
 def test_full_prefix_validation():

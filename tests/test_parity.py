@@ -75,6 +75,12 @@ def test_featuremap(dt, out_dt):
         assert_close(got, want, dict(rel_l2=5e-3, max_abs=4e-3), "phi")
     # each half of phi sums to 1
     np.testing.assert_allclose(got[..., :128].sum(-1), 1.0, atol=2e-2 if out_dt == torch.bfloat16 else 1e-5)
+    # the checked entry point: the same output, and a clean error word
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    phi2 = bha.featuremap(x, dev(c.W, act_dtype(c)), out_dtype=out_dt, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(phi2, phi)
 
 
 def test_featuremap_odd_dims_and_head_map():
