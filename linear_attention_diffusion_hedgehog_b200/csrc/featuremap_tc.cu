@@ -335,17 +335,9 @@ cudaError_t launch_featuremap_tc(const void* x, int T, int x_heads, int Hw, cons
   const int tiles = Hw * ((T + tok_per_tile - 1) / tok_per_tile);
   int nsm = device_sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
-  // fewest CTAs that finish in the same number of rounds, a multiple of Hw so each CTA keeps
-  // one W_g resident
-  const int rounds = (tiles + nsm - 1) / nsm;
-  int grid = (tiles + rounds - 1) / rounds;
-  if (Hw <= nsm) {
-    grid = (grid + Hw - 1) / Hw * Hw;
-    if (grid > nsm) grid = (nsm / Hw) * Hw;
-  } else {
-    grid = nsm;
-  }
-  if (grid > tiles) grid = tiles;
+  // fewest CTAs that finish in the least number of rounds, a multiple of Hw when that costs no
+  // round (each CTA then keeps one W_g resident)
+  const int grid = persistent_grid(tiles, Hw, nsm);
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(featuremap_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);

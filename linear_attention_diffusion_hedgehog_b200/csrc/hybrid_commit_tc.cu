@@ -809,18 +809,9 @@ cudaError_t launch_hybrid_commit_tc(const HybridArgs& a, float* S, float* Z, cud
   const int units = a.R * a.Hkv;
   int nsm = device_sm_count();
   if (nsm <= 0) return cudaErrorInvalidDevice;
-  // Fewest CTAs that still finish in the same number of rounds (every CTA then takes the
-  // same number of units and a larger share of the memory bandwidth), kept a multiple of Hkv
-  // so that each CTA stays on one KV head.
-  const int rounds = (units + nsm - 1) / nsm;
-  int grid = (units + rounds - 1) / rounds;
-  if (a.Hkv <= nsm) {
-    grid = (grid + a.Hkv - 1) / a.Hkv * a.Hkv;
-    if (grid > nsm) grid = (nsm / a.Hkv) * a.Hkv;
-  } else {
-    grid = nsm;
-  }
-  if (grid > units) grid = units;
+  // Fewest CTAs that still finish in the least number of rounds, a multiple of Hkv when that
+  // costs no round (each CTA then stays on one KV head).
+  const int grid = persistent_grid(units, a.Hkv, nsm);
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(hybrid_commit_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);

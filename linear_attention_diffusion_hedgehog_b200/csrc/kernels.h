@@ -110,6 +110,11 @@ enum TmaSwizzle { kTma128B, kTma128BAtom32, kTmaNone };
 bool make_tensor_map(CUtensorMap* m, bool f32, int rank, const void* base, const uint64_t* dims,
                      const uint64_t* strides_bytes, const uint32_t* box, TmaSwizzle swizzle);
 int device_sm_count();
+// Grid of a persistent kernel over `units` work units striding by the grid: the fewest CTAs
+// (at most nsm, one per SM) that finish in the least number of rounds, rounded up to a
+// multiple of stride_mult when that costs no extra round (each CTA then keeps one weight
+// matrix resident; otherwise it reloads the weights when the head changes).
+int persistent_grid(int units, int stride_mult, int nsm);
 
 // tensor-core kernels
 bool hybrid_tc_supports(const HybridArgs& a, bool act_bf16);

@@ -59,4 +59,14 @@ int device_sm_count() {
   return n;
 }
 
+int persistent_grid(int units, int stride_mult, int nsm) {
+  const int rounds = (units + nsm - 1) / nsm;
+  int grid = (units + rounds - 1) / rounds;
+  if (stride_mult > 1 && stride_mult <= nsm) {
+    const int g2 = (grid + stride_mult - 1) / stride_mult * stride_mult;
+    if (g2 <= nsm) grid = g2;
+  }
+  return grid < units ? grid : units;
+}
+
 }  // namespace bha
