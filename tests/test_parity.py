@@ -656,7 +656,7 @@ def _run_fused(c, S, Z, alpha=None, state_slot=None, dtype=None):
     return O
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(16, 4), (16, 16)])
+@pytest.mark.parametrize("Hq,Hkv", [(16, 4), (16, 8), (16, 16)])
 def test_fused_step_and_commit_ragged_slots_gate(Hq, Hkv):
     """The last step of a block with its commit in one call: ragged blocks (0, 1, 31, 32
     tokens), a permuted slot map, the gate and drawn states.  The output reads the states as
