@@ -12,17 +12,20 @@
 // cache in 128-key tiles:
 //   S_i   = Q K_i^T              bf16 MMA into one of two TMEM score buffers (the next
 //                                tile's scores are computed while this tile's softmax runs)
-//   P_i   = 2^{S_i log2e/sqrt d - m_i}   online softmax, one thread per row, P in bf16
-//   D_i   = P_i V_i              bf16 MMA into one of two TMEM buffers
-//   O     = O 2^{m_{i-1} - m_i} + D_i    in registers
-// With one split the unit writes O / l; with several, it writes the unnormalised O, the
-// running max m (log2 units) and the sum l to the workspace and a combine kernel merges the
-// splits.  Keys at or past kv_len are masked by index and their V rows are cleared in
-// shared memory, so whatever the cache holds there (even non-finite bytes) has no effect.
+//   P_i   = 2^{S_i log2e/sqrt d - m_ref}   online softmax, one thread per row, P in bf16
+//                                written to TMEM (two keys per column)
+//   O    += P_i V_i              bf16 MMA with P from TMEM, accumulating in a TMEM O
+// The reference max m_ref is raised only when a tile's row max exceeds it by more than
+// kTau (log2 units); only then is the row's O (and l) rescaled in place, between two P V
+// products, so P <= 2^kTau.  With one split the unit writes O / l; with several, it writes
+// the unnormalised O, m_ref and l to the workspace and a combine kernel merges the splits.
+// Keys at or past kv_len are masked by index and their V rows are cleared in shared memory,
+// so whatever the cache holds there (even non-finite bytes) has no effect.
 //
-// Roles (192 threads): warp 0 TMA producer (Q per unit, K/V tiles through a 2-stage ring),
-// warp 1 TMEM owner and MMA issuer, warps 2-5 softmax / accumulation / epilogue.  Every wait
-// is bounded; on expiry the CTA records BHA_ERR_TIMEOUT, drains, frees TMEM and returns.
+// Roles (192 threads): warp 0 TMA producer (Q per unit, K/V tiles through a 3-stage ring:
+// P lives in TMEM, so shared memory holds only Q and the ring), warp 1 TMEM owner and MMA
+// issuer, warps 2-5 softmax, rescaling and epilogue.  Every wait is bounded; on expiry the CTA
+// records BHA_ERR_TIMEOUT, drains, frees TMEM and returns.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -37,16 +40,20 @@ constexpr int kG = 4;
 constexpr int kBlk = 32;
 constexpr int kM = kG * kBlk;  // 128 query rows
 constexpr int kKT = 128;       // keys per tile
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kThreads = 192;
 
 constexpr uint32_t kQBytes = kM * kD * 2;    // 32 KiB: [d half][128 rows][128 B]
 constexpr uint32_t kTileBytes = kKT * kD * 2;  // 32 KiB: [d half][128 keys][128 B]
-constexpr uint32_t kPBytes = kM * kKT * 2;   // 32 KiB: [key half][128 rows][128 B]
 
 constexpr uint32_t kColS = 0;    // two score buffers, 128 columns each
-constexpr uint32_t kColD = 256;  // two P V buffers, 128 columns each
+constexpr uint32_t kColO = 256;  // the output accumulator O (128 columns), P V accumulates here
+constexpr uint32_t kColP = 384;  // P in bf16, two keys per column (64 columns), the A operand of P V
 constexpr uint32_t kTmemCols = 512;
+// Lazy rescaling: P is formed against a reference max m_ref that is raised only when a tile's
+// row max exceeds it by more than kTau (log2 units), so P <= 2^kTau and O, l are rescaled in
+// place only then.
+constexpr float kTau = 8.f;
 
 constexpr uint32_t kIdQK = tc::instr_desc(1, 0, 0, kM, kKT);
 constexpr uint32_t kIdPV = tc::instr_desc(1, 0, 1, kM, kD);
@@ -55,9 +62,8 @@ struct __align__(1024) Smem {
   uint8_t q[kQBytes];
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
-  uint8_t p[kPBytes];
   uint64_t q_full, q_empty, kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_free[2], d_full[2], d_free[2], p_full, p_free, drain;
+  uint64_t s_full[2], s_free[2], p_full, pv_done, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -107,11 +113,9 @@ __global__ void __launch_bounds__(kThreads, 1) full_prefix_tc_kernel(const __gri
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&sm.s_full[i], 1);
       tc::mbar_init(&sm.s_free[i], 4);
-      tc::mbar_init(&sm.d_full[i], 1);
-      tc::mbar_init(&sm.d_free[i], 4);
     }
     tc::mbar_init(&sm.p_full, 4);
-    tc::mbar_init(&sm.p_free, 1);
+    tc::mbar_init(&sm.pv_done, 1);
     tc::mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     tc::fence_barrier_init();
@@ -168,22 +172,20 @@ __global__ void __launch_bounds__(kThreads, 1) full_prefix_tc_kernel(const __gri
     if (lane == 0) {
       int qk = 0, gt = 0;
       bool ok = true, issued = false;
-      auto issue_pv = [&](int tile) -> bool {
-        // P_tile V_tile into D buffer (tile & 1)
-        const int db = tile & 1, st = tile % kStages;
+      // O (+)= P_tile V_tile: the first tile of a unit overwrites O, the others accumulate
+      // (the softmax warps rescale O in place, between two of these, when m_ref rises)
+      auto issue_pv = [&](int tile, bool first) -> bool {
+        const int st = tile % kStages;
         if (!tc::mbar_wait(&sm.p_full, tile & 1, abort_flag, lim)) return false;
-        if (tile >= 2 && !tc::mbar_wait(&sm.d_free[db], ((tile >> 1) - 1) & 1, abort_flag, lim)) return false;
         tc::tc_fence_after();
-        const uint32_t pa = tc::smem_u32(sm.p), va = tc::smem_u32(sm.v[st]);
+        const uint32_t va = tc::smem_u32(sm.v[st]);
 #pragma unroll
         for (int kk = 0; kk < kKT / 16; ++kk) {
-          const uint64_t a = tc::smem_desc(pa + (kk >> 2) * (kPBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
           const uint64_t b = tc::smem_desc(va + kk * 2048, kTileBytes / 2, 1024, tc::kSwizzle128B);
-          tc::mma_bf16_ss(tbase + kColD + db * 128, a, b, kIdPV, kk > 0);
+          tc::mma_bf16_ts(tbase + kColO, tbase + kColP + kk * 8, b, kIdPV, (first && kk == 0) ? 0u : 1u);
         }
-        tc::mma_commit(&sm.d_full[db]);
+        tc::mma_commit(&sm.pv_done);
         tc::mma_commit(&sm.kv_empty[st]);
-        tc::mma_commit(&sm.p_free);
         return true;
       };
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
@@ -207,10 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1) full_prefix_tc_kernel(const __gri
           tc::mma_commit(&sm.s_full[sb]);
           if (i == x.nt - 1) tc::mma_commit(&sm.q_empty);
           issued = true;
-          if (i >= 1 && !issue_pv(gt - 1)) { ok = false; break; }
+          if (i >= 1 && !issue_pv(gt - 1, i == 1)) { ok = false; break; }
         }
         if (!ok) break;
-        if (!issue_pv(gt - 1)) { ok = false; break; }
+        if (!issue_pv(gt - 1, x.nt == 1)) { ok = false; break; }
       }
       if (issued) {
         volatile int never = 0;
@@ -231,27 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1) full_prefix_tc_kernel(const __gri
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
       Unit x;
       if (!decode_unit(p, u, false, &x)) continue;
-      float o[kD];
-#pragma unroll
-      for (int c = 0; c < kD; ++c) o[c] = 0.f;
-      float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
-      auto accumulate = [&](int tile, float alpha) -> bool {
-        const int db = tile & 1;
-        if (!tc::mbar_wait(&sm.d_full[db], (tile >> 1) & 1, abort_flag, lim)) return false;
-        tc::tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < kD / 32; ++c) {
-          float dv[32];
-          tc::tmem_ld32(tl + kColD + db * 128 + c * 32, dv);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], alpha, dv[i]);
-        }
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&sm.d_free[db]);
-        return true;
-      };
+      // m_ref: the reference max P is formed against (log2 units); l: sum of P against it
+      float m = -INFINITY, l = 0.f;
       for (int i = 0; i < x.nt; ++i, ++gt) {
         const int sb = gt & 1, st = gt % kStages;
         if (!tc::mbar_wait(&sm.s_full[sb], (gt >> 1) & 1, abort_flag, lim)) { ok = false; break; }
@@ -259,52 +242,59 @@ __global__ void __launch_bounds__(kThreads, 1) full_prefix_tc_kernel(const __gri
         const int key0 = (x.t0 + i) * kKT;
         const int valid_keys = min(kKT, x.L - key0);
         const uint32_t scol = tl + kColS + sb * 128;
-        // pass 1: row max of this tile's scaled scores (keys at or past kv_len excluded)
+        // the row's 128 scores of this tile, scaled to log2 units; keys at or past kv_len -inf
+        float sv[kKT];
+#pragma unroll
+        for (int c = 0; c < kKT / 32; ++c) tc::tmem_ld32(scol + c * 32, *reinterpret_cast<float(*)[32]>(sv + c * 32));
+        tc::tmem_wait_ld();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&sm.s_free[sb]);  // the score buffer may be refilled
         float tmax = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < kKT / 32; ++c) {
-          float tmp[32];
-          tc::tmem_ld32(scol + c * 32, tmp);
-          tc::tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (c * 32 + j < valid_keys) tmax = fmaxf(tmax, tmp[j] * scale_log2);
+        for (int j = 0; j < kKT; ++j) {
+          sv[j] = j < valid_keys ? sv[j] * scale_log2 : -INFINITY;
+          tmax = fmaxf(tmax, sv[j]);
         }
-        const float m_new = fmaxf(m, tmax);
-        const float alpha = (m_new == -INFINITY) ? 1.f : tc::ex2(m - m_new);
-        // P is free once the previous tile's P V has completed
-        if (gt >= 1 && !tc::mbar_wait(&sm.p_free, (gt - 1) & 1, abort_flag, lim)) { ok = false; break; }
-        // pass 2: P = 2^{s - m_new} in bf16; keys [64 a, 64 a + 64) in atom a, 16-byte chunk c
-        // of a row at chunk c ^ (row % 8)
-        float psum = 0.f;
+        // the P buffer (and O) are free once the previous tile's P V has completed
+        if (gt >= 1 && !tc::mbar_wait(&sm.pv_done, (gt - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        tc::tc_fence_after();
+        if (i == 0) {
+          m = tmax;  // every tile of a split holds at least one key below kv_len
+        } else if (tmax > m + kTau) {
+          // raise m_ref: O and l are rescaled in place before this tile's P V accumulates
+          const float alpha = tc::ex2(m - tmax);
 #pragma unroll 1
-        for (int c = 0; c < kKT / 32; ++c) {
-          float tmp[32];
-          tc::tmem_ld32(scol + c * 32, tmp);
-          tc::tmem_wait_ld();
-          uint32_t pk[16];
+          for (int c = 0; c < kD / 32; ++c) {
+            float ov[32];
+            tc::tmem_ld32(tl + kColO + c * 32, ov);
+            tc::tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const bool v0 = c * 32 + j < valid_keys, v1 = c * 32 + j + 1 < valid_keys;
-            const float a0 = v0 ? tc::ex2(fmaf(tmp[j], scale_log2, -m_new)) : 0.f;
-            const float a1 = v1 ? tc::ex2(fmaf(tmp[j + 1], scale_log2, -m_new)) : 0.f;
+            for (int j = 0; j < 32; ++j) ov[j] *= alpha;
+            tc::tmem_st32(tl + kColO + c * 32, ov);
+          }
+          tc::tmem_wait_st();
+          l *= alpha;
+          m = tmax;
+        }
+        // P = 2^{s - m_ref} in bf16, two keys per TMEM column (the A operand of P V)
+        float psum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int j = 0; j < 64; j += 2) {
+            const float a0 = tc::ex2(sv[c * 64 + j] - m);   // 2^-inf = 0 for masked keys
+            const float a1 = tc::ex2(sv[c * 64 + j + 1] - m);
             const __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
             psum += __low2float(b2) + __high2float(b2);
             pk[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
           }
-          uint8_t* prow = sm.p + (c >> 1) * (kPBytes / 2) + row * 128;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int ch = (c & 1) * 4 + q4;
-            *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
-                make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-          }
+          tc::tmem_st16u(tl + kColP + c * 32, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+          tc::tmem_st16u(tl + kColP + c * 32 + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
         }
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&sm.s_free[sb]);
-        l = l * alpha + psum;
-        m = m_new;
+        tc::tmem_wait_st();
+        l += psum;
         if (valid_keys < kKT) {
           // V rows past kv_len are cleared (the cache may hold anything there)
           const int per_half = (kKT - valid_keys) * 8;
@@ -315,13 +305,27 @@ __global__ void __launch_bounds__(kThreads, 1) full_prefix_tc_kernel(const __gri
           }
         }
         tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&sm.p_full);
-        if (i >= 1 && !accumulate(gt - 1, alpha_prev)) { ok = false; break; }
-        alpha_prev = alpha;
       }
       if (!ok) break;
-      if (x.nt > 0 && !accumulate(gt - 1, alpha_prev)) { ok = false; break; }
+      // O of this unit is complete once its last P V has
+      if (x.nt > 0) {
+        if (!tc::mbar_wait(&sm.pv_done, (gt - 1) & 1, abort_flag, lim)) { ok = false; break; }
+        tc::tc_fence_after();
+      }
+      float o[kD];
+#pragma unroll
+      for (int c = 0; c < kD / 32; ++c) {
+        if (x.nt > 0) {
+          tc::tmem_ld32(tl + kColO + c * 32, *reinterpret_cast<float(*)[32]>(o + c * 32));
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[c * 32 + j] = 0.f;
+        }
+      }
+      tc::tmem_wait_ld();
       // epilogue
       if (t < x.n) {
         const size_t orow = (size_t)(x.lo + t) * p.Hq + kG * x.g + hl;
