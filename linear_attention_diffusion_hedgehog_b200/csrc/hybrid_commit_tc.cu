@@ -527,7 +527,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
       // Scale of the linear branch (log2 units).  Both branches meet in A+ with P stored as
       // w 2^{s_j} sum e+, so e+ and e- are shifted down by tl = max(0, m - 100): then every
       // stored P is below 2^{107} and no e exceeds 1, and when m > 100 the linear branch,
-      // which tl makes smaller still, is in any case below 2^{-90} of the softmax branch.
+      // which tl makes smaller still, is in any case below 2^{-90} of the softmax branch (if
+      // the shift flushes every e+ and e- to 0, P is formed as if sum e+ were 2^{-tl}).
       // States that are all zero (no committed block) add nothing: e+ = e- = 0 and P is
       // shifted by m instead, so a block whose scores are all very negative stays exact.
       float zmax;
@@ -590,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
           // buffer is free once V has landed (V is reloaded only after the previous P V has
           // completed).
           vgood = __all_sync(0xffffffffu, tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim));
-          const float lsp = lin ? tc::lg2(esp) : -m2;
+          const float lsp = lin ? (esp > 0.f ? tc::lg2(esp) : -tl2) : -m2;
           float sv[32];
           tc::tmem_ld32(tl + kColS, sv);
           tc::tmem_wait_ld();
@@ -643,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
       const int fb = k & 1;
       if (k >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(&sm.fin_empty[fb], ((k - 2) >> 1) & 1, abort_flag, lim)))
         break;
-      const float rpm = lin ? esp / esm : 0.f;
+      const float rpm = lin && esm > 0.f ? esp / esm : 0.f;
       const float den = psum + (lin ? zsp + zsm * rpm : 0.f);
       const float inv = den != 0.f ? 1.f / den : 0.f;
       sm.fin[fb][0][row] = inv;

@@ -13,6 +13,10 @@ from linear_attention_diffusion_hedgehog_b200 import bha
 
 TOL_BF16 = dict(max_abs=2e-2, rel_l2=5e-3)
 TOL_F32 = dict(rel_l2=1e-5, rel_max=1e-5)
+# States built from hundreds to thousands of tokens: the stated relative L2 bound, and the
+# largest error relative to the largest entry held to the same level (the absolute 2e-2 bound
+# is stated for outputs and for the 32-commit states of the block-commit workload)
+TOL_STATE_LONG = dict(rel_l2=5e-3, rel_max=5e-3)
 
 
 def dev(x, dtype):

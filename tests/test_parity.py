@@ -6,8 +6,8 @@ import torch
 
 from linear_attention_diffusion_hedgehog_b200 import bha, inputs
 from oracle import bha_ref as ref
-from tests.gpu_util import (TOL_BF16, TOL_F32, act_dtype, assert_close, build_states_on_gpu,
-                            dev, host64)
+from tests.gpu_util import (TOL_BF16, TOL_F32, TOL_STATE_LONG, act_dtype, assert_close,
+                            build_states_on_gpu, dev, host64)
 
 pytestmark = pytest.mark.gpu
 
@@ -543,12 +543,13 @@ def test_bounded_wait_gives_up_and_reports_timeout():
 
 # ------------------------------------------------------------------- extreme block logits
 
-def _extreme_logit_case(sign, aligned_all, prefix, seed, dtype="bf16", d=128, F=256, Hq=16, Hkv=4):
-    """Block scores near sign * 100 (natural units).  aligned_all: every key of a request is
+def _extreme_logit_case(sign, aligned_all, prefix, seed, dtype="bf16", d=128, F=256, Hq=16, Hkv=4,
+                        level=100.0):
+    """Block scores near sign * level (natural units).  aligned_all: every key of a request is
     close to one direction v0 and every query is sign * v0, so all of a row's scores are about
-    sign * 100; otherwise each query copies one key of its block (scaled by sign), so one score
-    per row is about sign * 100 and the rest are O(25).  prefix: states drawn from 700-token
-    prefixes, or all zero."""
+    sign * level; otherwise each query copies one key of its block (scaled by sign), so one
+    score per row is about sign * level and the rest are O(level / 4).  prefix: states drawn
+    from 700-token prefixes, or all zero."""
     lens = [32, 17, 1, 32]
     c = inputs.decode_case(R=4, Hq=Hq, Hkv=Hkv, d=d, F=F, block_lens=lens, prefix_lens=0,
                            seed=seed, dtype=dtype)
@@ -557,7 +558,7 @@ def _extreme_logit_case(sign, aligned_all, prefix, seed, dtype="bf16", d=128, F=
     G = Hq // Hkv
     K = np.empty_like(c.K)
     Q = np.empty_like(c.Q)
-    amp = np.sqrt(100.0 * np.sqrt(d) / d)  # |q| |k| / sqrt d ~ 100 for unit-variance directions
+    amp = np.sqrt(level * np.sqrt(d) / d)  # |q| |k| / sqrt d ~ level for unit-variance directions
     for r in range(4):
         lo, hi = c.cu_blk[r], c.cu_blk[r + 1]
         for g in range(Hkv):
@@ -578,23 +579,42 @@ def _extreme_logit_case(sign, aligned_all, prefix, seed, dtype="bf16", d=128, F=
     return c, S_np, Z_np
 
 
-@pytest.mark.parametrize("sign,aligned_all,prefix", [
-    (+1, False, False), (+1, False, True), (+1, True, False), (+1, True, True),
-    (-1, True, False), (-1, True, True)])
-def test_decode_step_extreme_block_logits(sign, aligned_all, prefix):
+@pytest.mark.parametrize("sign,aligned_all,prefix,level", [
+    (+1, False, False, 100), (+1, False, True, 100), (+1, True, False, 100), (+1, True, True, 100),
+    (-1, True, False, 100), (-1, True, True, 100), (+1, True, True, 180), (+1, False, True, 180)])
+def test_decode_step_extreme_block_logits(sign, aligned_all, prefix, level):
     """Scores of about +100 overflow exp in fp32 unless shifted, and a row whose scores are
     all about -100 underflows it: with an empty prefix the output must still be the block
-    softmax, with a prefix the linear branch must dominate (softmax weight ~e^-100); checked
-    against the float64 oracle on the tensor-core path."""
-    c, S_np, Z_np = _extreme_logit_case(sign, aligned_all, prefix, seed=50 + 7 * aligned_all + 3 * prefix)
+    softmax, with a prefix the linear branch must dominate (softmax weight ~e^-100).  At +180
+    the shift that keeps P finite flushes every linear-branch exponential to 0 and the output
+    is the block softmax.  Checked against the float64 oracle on the tensor-core path."""
+    c, S_np, Z_np = _extreme_logit_case(sign, aligned_all, prefix, seed=50 + 7 * aligned_all + 3 * prefix,
+                                        level=float(level))
     d = bha.make_dims(4, 16, 4, 128, 256, 32, int(c.cu_blk[-1]), 4, torch.bfloat16)
     assert bha.kernel_variant(d, 1) == 1
     s = np.einsum("thd,tgd->th", c.Q.reshape(-1, 4, 4, 128).astype(np.float64)[:, :, 0, :],
                   c.K.astype(np.float64)) / np.sqrt(128.0)
-    assert np.abs(s).max() > 80  # the case really reaches the edge
+    assert np.abs(s).max() > 0.8 * level  # the case really reaches the edge
     O = run_hybrid(c, dev(S_np, torch.float32), dev(Z_np, torch.float32))
     want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, S_np.astype(np.float64), Z_np.astype(np.float64), c.W)
     assert_close(host64(O), want, TOL_BF16, "O")
+
+
+@pytest.mark.parametrize("aligned_all,level", [(True, 180), (False, 100)])
+def test_fused_step_and_commit_extreme_block_logits(aligned_all, level):
+    """The fused step and commit at the same edges (states from 700-token prefixes, scores of
+    about +level): the output against the oracle's step, the states (entries of up to ~40, the
+    size of long-prefix states) against its commit."""
+    c, S_np, Z_np = _extreme_logit_case(+1, aligned_all, True, seed=57 + 7 * aligned_all, level=float(level))
+    d = bha.make_dims(4, 16, 4, 128, 256, 32, int(c.cu_blk[-1]), 4, torch.bfloat16)
+    assert bha.kernel_variant(d, 4) == 1
+    S, Z = dev(S_np, torch.float32), dev(Z_np, torch.float32)
+    O = _run_fused(c, S, Z)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, S_np.astype(np.float64), Z_np.astype(np.float64), c.W)
+    assert_close(host64(O), want, TOL_BF16, "O")
+    So, Zo = ref.commit_block(c.cu_blk, c.K, c.V, c.W, S_np.astype(np.float64), Z_np.astype(np.float64))
+    assert_close(host64(S), So, TOL_STATE_LONG, "S")
+    assert_close(host64(Z), Zo, TOL_STATE_LONG, "Z")
 
 
 @pytest.mark.parametrize("sign,prefix", [(+1, False), (+1, True), (-1, False), (-1, True)])
