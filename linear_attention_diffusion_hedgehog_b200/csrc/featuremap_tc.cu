@@ -14,15 +14,16 @@
 // Roles (320 threads):
 //   warp 0      TMA producer: W_g when it changes, x tiles through a 2-stage ring.
 //   warp 1      TMEM owner and MMA issuer: u of tile k into TMEM buffer k % 2 (two buffers of
-//               256 columns: u, overwritten in place by e+, then e-), so the next tile's MMA
+//               256 columns: u, then e- in place, and e+ beside it), so the next tile's MMA
 //               overlaps this tile's epilogue.
 //   warps 2-9   two groups of four, taking alternate tiles (warps 2-5 the even ones, 6-9 the
 //               odd ones, matching the TMEM buffers), so one group's exponentials overlap the
 //               other group's read-out and stores.  In a group, warp wq owns TMEM lane quarter
-//               wq and each thread one whole row: max and min of its 128 u values, e+ and e-
-//               written to TMEM with their sums, then read back normalised, 32 rows x 128
-//               bytes at a time, into a double-buffered staging slot that one asynchronous
-//               bulk tensor store writes to phi.
+//               wq and each thread one whole row: max and min of its 128 u values; e+ written
+//               beside u with its sum and read back normalised, 32 rows x 128 bytes at a time,
+//               into a double-buffered staging slot that one asynchronous bulk tensor store
+//               writes to phi; then e- over u in place, likewise.  Storing phi+ before e- is
+//               computed halves the time from a tile's u to its first store.
 //
 // Every wait is bounded.  On expiry the CTA stops early, the call's output is undefined and
 // BHA_ERR_TIMEOUT goes to dev_err when the caller passed one; nothing traps and TMEM is freed.
@@ -44,7 +45,7 @@ constexpr uint32_t kXBytes = kM * kD * 2;      // 32 KiB: [d half][128 rows][128
 constexpr uint32_t kWBytes = kD * kFh * 2;     // 32 KiB: [f half][128 rows of d][128 B]
 constexpr uint32_t kStgBytes = 32 * 128;       // 4 KiB: 32 rows x 128 bytes
 
-constexpr uint32_t kTmemCols = 512;            // two buffers of [u / e+ (128) | e- (128)]
+constexpr uint32_t kTmemCols = 512;            // two buffers of [u / e- (128) | e+ (128)]
 constexpr uint32_t kIdXW = tc::instr_desc(1, 0, 1, kM, kFh);  // bf16, B MN-major
 
 struct __align__(1024) Smem {
@@ -200,84 +201,94 @@ __global__ void __launch_bounds__(kThreads, 1) featuremap_tc_kernel(const __grid
           mn = fminf(mn, fminf(u0[i], u1[i]));
         }
       }
-      // unnormalised e+ over u in place and e- beside it, with their sums
+      // phi, 32 rows x 128 bytes per store: fp32 in chunks of 32 columns, bf16 in chunks of
+      // 64; half 0 (phi+) is stored while half 1's exponentials are computed
+      const int tok_w = t0 + row0 / p.G;       // first token of this warp's rows
+      const int head_w = g * p.G + row0 % p.G;  // first head of this warp's rows
+      const bool store = tok_w < p.T;
+      const int nchunks = p.out_bf16 ? 2 : 4;  // per half
+      // normalised read-out of one half (e at TMEM column src), one bulk store per chunk
+      auto readout = [&](const int half, const uint32_t src, const float sc, const bool last) {
+        for (int c = 0; c < nchunks; ++c) {
+          uint32_t packed[32];
+          int f0;  // first phi column of the chunk
+          if (p.out_bf16) {
+            float a[32], bb[32];
+            tc::tmem_ld32(tb + src + c * 64, a);
+            tc::tmem_ld32(tb + src + c * 64 + 32, bb);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              packed[i] = pack_bf16(a[2 * i] * sc, a[2 * i + 1] * sc);
+              packed[16 + i] = pack_bf16(bb[2 * i] * sc, bb[2 * i + 1] * sc);
+            }
+            f0 = half * kFh + c * 64;
+          } else {
+            float a[32];
+            tc::tmem_ld32(tb + src + c * 32, a);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) packed[i] = __float_as_uint(a[i] * sc);
+            f0 = half * kFh + c * 32;
+          }
+          if (last && c == nchunks - 1) {
+            // every TMEM read of this tile is done: the MMA may refill the buffer
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sm.tm_empty[b]);
+          }
+          // staging slot nst % 2: its previous store (two stores ago) must have read it
+          uint8_t* slot = sm.stg[sw][nst & 1];
+          if (lane == 0) bulk_wait_read_one();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4*>(slot + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+          if (store) {
+            if (lane == 0) {
+              tc::tma_store_3d(&p.tm_o, slot, f0, head_w, tok_w);
+              tc::bulk_commit();
+            }
+            ++nst;
+          }
+        }
+      };
+
+      // e+ (unnormalised) into columns 128.. with its sum, then phi+ stored from there
       const float bpl = mx * log2e, bml = mn * log2e;
       float esp = 0.f, esm = 0.f;
 #pragma unroll 1
       for (int c = 0; c < kFh / 32; ++c) {
-        float uu[32], ep[32];
+        float uu[32];
         tc::tmem_ld32(tb + c * 32, uu);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float a = uu[i] * log2e;
-          ep[i] = tc::ex2(a - bpl);
-          uu[i] = tc::ex2(bml - a);
-          esp += ep[i];
-          esm += uu[i];
+          uu[i] = tc::ex2(uu[i] * log2e - bpl);
+          esp += uu[i];
         }
-        tc::tmem_st32(tb + c * 32, ep);
         tc::tmem_st32(tb + 128 + c * 32, uu);
       }
       tc::tmem_wait_st();
-      const float ip = 1.f / esp, im = 1.f / esm;
-
-      // phi, 32 rows x 128 bytes per store: fp32 in eight chunks of 32 columns (e+ then e-),
-      // bf16 in four chunks of 64 columns
-      const int tok_w = t0 + row0 / p.G;       // first token of this warp's rows
-      const int head_w = g * p.G + row0 % p.G;  // first head of this warp's rows
-      const bool store = tok_w < p.T;
-      const int nchunks = p.out_bf16 ? 4 : 8;
-      for (int c = 0; c < nchunks; ++c) {
-        uint32_t packed[32];
-        int f0;  // first phi column of the chunk
-        if (p.out_bf16) {
-          const int half = c >> 1, cc = c & 1;  // 64 columns of e+ or e-
-          const float sc = half ? im : ip;
-          float a[32], bb[32];
-          tc::tmem_ld32(tb + half * 128 + cc * 64, a);
-          tc::tmem_ld32(tb + half * 128 + cc * 64 + 32, bb);
-          tc::tmem_wait_ld();
+      readout(0, 128, 1.f / esp, false);
+      // e- over u in place with its sum, then phi- stored from there
+#pragma unroll 1
+      for (int c = 0; c < kFh / 32; ++c) {
+        float uu[32];
+        tc::tmem_ld32(tb + c * 32, uu);
+        tc::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            packed[i] = pack_bf16(a[2 * i] * sc, a[2 * i + 1] * sc);
-            packed[16 + i] = pack_bf16(bb[2 * i] * sc, bb[2 * i + 1] * sc);
-          }
-          f0 = half * kFh + cc * 64;
-        } else {
-          const int half = c >> 2, cc = c & 3;  // 32 columns of e+ or e-
-          const float sc = half ? im : ip;
-          float a[32];
-          tc::tmem_ld32(tb + half * 128 + cc * 32, a);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) packed[i] = __float_as_uint(a[i] * sc);
-          f0 = half * kFh + cc * 32;
+        for (int i = 0; i < 32; ++i) {
+          uu[i] = tc::ex2(bml - uu[i] * log2e);
+          esm += uu[i];
         }
-        if (c == nchunks - 1) {
-          // every TMEM read of this tile is done: the MMA may refill the buffer
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&sm.tm_empty[b]);
-        }
-        // staging slot nst % 2: its previous store (two stores ago) must have read it
-        uint8_t* slot = sm.stg[sw][nst & 1];
-        if (lane == 0) bulk_wait_read_one();
-        __syncwarp();
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<uint4*>(slot + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-              make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-        tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (store) {
-          if (lane == 0) {
-            tc::tma_store_3d(&p.tm_o, slot, f0, head_w, tok_w);
-            tc::bulk_commit();
-          }
-          ++nst;
-        }
+        tc::tmem_st32(tb + c * 32, uu);
       }
+      tc::tmem_wait_st();
+      readout(1, 0, 1.f / esm, true);
     }
     if (lane == 0) tc::bulk_wait_all();
   }
