@@ -93,7 +93,7 @@ struct __align__(1024) Smem {
   uint64_t q_full, k_full, qk_empty, v_full, v_empty, v_ready, z_full[2], z_empty[2];
   uint64_t s_full[kStages], s_empty[kStages];
   uint64_t e_ready[kGroups], p_ready;
-  uint64_t w_full, u_full, acc_full, acc_empty, drain, fin_full[2], fin_empty[2];
+  uint64_t w_full, u_full, s_ready, acc_full, acc_empty, drain, fin_full[2], fin_empty[2];
   uint64_t uk_done, u_staged, phi_ready, ds_full, ds_empty, commit_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -238,6 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
     tc::mbar_init(&sm.p_ready, 4);
     tc::mbar_init(&sm.w_full, 1);
     tc::mbar_init(&sm.u_full, 1);
+    tc::mbar_init(&sm.s_ready, 1);
     tc::mbar_init(&sm.acc_full, 1);
     tc::mbar_init(&sm.acc_empty, 4);  // the four epilogue warps
     tc::mbar_init(&sm.drain, 1);
@@ -385,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
       const uint32_t qa = tc::smem_u32(sm.q);
       const uint32_t ka = tc::smem_u32(sm.k);
       const uint32_t phia = tc::smem_u32(sm.s[kCommitStage][0]);    // phi of the block
-      // u = Q W_g and s = Q K^T of unit j
+      // s = Q K^T, then u = Q W_g of unit j
       auto issue_uqk = [&](const Unit& y, int j) -> bool {
         if (y.g != g_res) {
           if (!tc::mbar_wait(&sm.w_full, w_seen & 1, abort_flag, lim)) return false;
@@ -398,14 +399,15 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t a = tc::smem_desc(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
-          const uint64_t b = tc::smem_desc(wa + kk * 2048, kWBytes / 2, 1024, tc::kSwizzle128B);
-          tc::mma_bf16_ss(tbase + kColU, a, b, kIdQW, kk > 0);
+          const uint64_t b = tc::smem_desc(ka + (kk >> 2) * (kKBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
+          tc::mma_bf16_ss(tbase + kColS, a, b, kIdQK, kk > 0);
         }
+        tc::mma_commit(&sm.s_ready);  // the feature map starts on the scores
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t a = tc::smem_desc(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
-          const uint64_t b = tc::smem_desc(ka + (kk >> 2) * (kKBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
-          tc::mma_bf16_ss(tbase + kColS, a, b, kIdQK, kk > 0);
+          const uint64_t b = tc::smem_desc(wa + kk * 2048, kWBytes / 2, 1024, tc::kSwizzle128B);
+          tc::mma_bf16_ss(tbase + kColU, a, b, kIdQW, kk > 0);
         }
         tc::mma_commit(&sm.u_full);
         tc::mma_commit(&sm.qk_empty);
@@ -505,7 +507,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
     int ucur = blockIdx.x;
     Unit x{};
     for (int k = 0; next_unit(p, units, &ucur, false, &x); ++k) {
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim))) break;
+      // the block scores first (u is still being computed behind them)
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.s_ready, k & 1, abort_flag, lim))) break;
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.z_full[k & 1], (k >> 1) & 1, abort_flag, lim))) break;
       tc::tc_fence_after();
 
@@ -542,6 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
       const float tl2 = lin ? fmaxf(0.f, m2 - 100.f) : INFINITY;
 
       // max and min of u over the row's 128 features
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim))) break;
+      tc::tc_fence_after();
       float mx = -INFINITY, mn = INFINITY;
 #pragma unroll 1
       for (int c = 0; c < kGroups; c += 2) {

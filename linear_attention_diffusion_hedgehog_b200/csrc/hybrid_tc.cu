@@ -36,11 +36,12 @@
 //               atoms, the layout a tf32 MN-major operand needs) through a 4-stage ring that
 //               holds one whole unit, with V issued ahead of the last stage.
 //   warp 1      TMEM owner and MMA issuer (one thread), per unit k: A+ += e+ S+ and
-//               A- += e- S- group by group (tf32, e from TMEM), then u = Q W_g and s = Q K^T of
-//               unit k+1 (bf16), then A+ += P V of unit k (bf16).  MMAs of one thread execute
-//               in issue order, so unit k+1's u and s overwrite e+ and the top of e- only after
-//               unit k's e S has read them, and unit k+1's feature map can start while unit k's
-//               P V is still waiting for its P.
+//               A- += e- S- group by group (tf32, e from TMEM), then s = Q K^T and u = Q W_g of
+//               unit k+1 (bf16, each announced on its own barrier, so that the feature map
+//               takes the row max of the scores while u is computed), then A+ += P V of unit k
+//               (bf16).  MMAs of one thread execute in issue order, so unit k+1's s and u
+//               overwrite the top of e- and e+ only after unit k's e S has read them, and unit
+//               k+1's feature map can start while unit k's P V is still waiting for its P.
 //   warps 2-5   feature map, one warp per TMEM lane quarter and one thread per tile row (its
 //               own TMEM lane): block-softmax max, e+ / e- group by group (each group released
 //               to the MMA as soon as the four warps have written it), P from the scores just
@@ -104,7 +105,7 @@ struct __align__(1024) Smem {
   uint64_t qk_full, qk_empty, v_full, v_empty, v_ready, z_full[2], z_empty[2];
   uint64_t s_full[kStages], s_empty[kStages];
   uint64_t e_ready[kGroups], p_ready;
-  uint64_t w_full, u_full, acc_full, acc_empty, drain, fin_full[2], fin_empty[2];
+  uint64_t w_full, u_full, s_ready, acc_full, acc_empty, drain, fin_full[2], fin_empty[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -171,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
     tc::mbar_init(&sm.p_ready, 4);
     tc::mbar_init(&sm.w_full, 1);
     tc::mbar_init(&sm.u_full, 1);
+    tc::mbar_init(&sm.s_ready, 1);
     tc::mbar_init(&sm.acc_full, 1);
     tc::mbar_init(&sm.acc_empty, 4);  // the four epilogue warps
     tc::mbar_init(&sm.drain, 1);
@@ -265,11 +267,11 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per unit k: A+/- += e S group by group, then the next unit's u and s, then A+ += P V.
-    // Issuing u(k+1) ahead of P V(k) lets the feature map of unit k+1 start as soon as the
-    // tensor pipe has finished e S(k), not after P V(k), which waits for unit k's P.  MMAs of
-    // one thread execute in issue order, so u(k+1) and s(k+1) overwrite e+ and the top of e-
-    // only after e S(k) has read them.
+    // Per unit k: A+/- += e S group by group, then the next unit's s and u, then A+ += P V.
+    // Issuing s(k+1) and u(k+1) ahead of P V(k) lets the feature map of unit k+1 start as soon
+    // as the tensor pipe has finished e S(k), not after P V(k), which waits for unit k's P.
+    // MMAs of one thread execute in issue order, so s(k+1) and u(k+1) overwrite the top of e-
+    // and e+ only after e S(k) has read them.
     if (lane == 0) {
       int g_res = -1, q = 0;
       uint32_t w_seen = 0;
@@ -279,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
       const uint32_t wa = tc::smem_u32(sm.w);
       const uint32_t qa = tc::smem_u32(sm.q);
       const uint32_t ka = tc::smem_u32(sm.k);
-      // u = Q W_g and s = Q K^T of unit j
+      // s = Q K^T, then u = Q W_g of unit j
       auto issue_uqk = [&](const Unit& y, int j) -> bool {
         if (y.g != g_res) {
           if (!tc::mbar_wait(&sm.w_full, w_seen & 1, abort_flag, lim)) return false;
@@ -291,14 +293,15 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t a = tc::smem_desc(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
-          const uint64_t b = tc::smem_desc(wa + kk * 2048, kWBytes / 2, 1024, tc::kSwizzle128B);
-          tc::mma_bf16_ss(tbase + kColU, a, b, kIdQW, kk > 0);
+          const uint64_t b = tc::smem_desc(ka + (kk >> 2) * (kKBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
+          tc::mma_bf16_ss(tbase + kColS, a, b, kIdQK, kk > 0);
         }
+        tc::mma_commit(&sm.s_ready);  // the feature map starts on the scores
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint64_t a = tc::smem_desc(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
-          const uint64_t b = tc::smem_desc(ka + (kk >> 2) * (kKBytes / 2) + (kk & 3) * 32, 16, 1024, tc::kSwizzle128B);
-          tc::mma_bf16_ss(tbase + kColS, a, b, kIdQK, kk > 0);
+          const uint64_t b = tc::smem_desc(wa + kk * 2048, kWBytes / 2, 1024, tc::kSwizzle128B);
+          tc::mma_bf16_ss(tbase + kColU, a, b, kIdQW, kk > 0);
         }
         tc::mma_commit(&sm.u_full);
         tc::mma_commit(&sm.qk_empty);
@@ -371,7 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
     int ucur = blockIdx.x;
     Unit x{};
     for (int k = 0; next_unit(p, units, &ucur, false, &x); ++k) {
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim))) break;
+      // the block scores first (u is still being computed behind them)
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.s_ready, k & 1, abort_flag, lim))) break;
       if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.z_full[k & 1], (k >> 1) & 1, abort_flag, lim))) break;
       tc::tc_fence_after();
 
@@ -408,6 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
       const float tl2 = lin ? fmaxf(0.f, m2 - 100.f) : INFINITY;
 
       // max and min of u over the row's 128 features
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&sm.u_full, k & 1, abort_flag, lim))) break;
+      tc::tc_fence_after();
       float mx = -INFINITY, mn = INFINITY;
 #pragma unroll 1
       for (int c = 0; c < kGroups; c += 2) {
