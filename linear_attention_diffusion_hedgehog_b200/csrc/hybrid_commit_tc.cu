@@ -703,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.fin_empty[fb]);
       __nv_bfloat16* orow = p.O + ((size_t)(x.lo + tok) * p.Hq + p.G * x.g + hl) * kD;
-      const bool live = tok < x.n;
+      const bool live = tok < x.n, o32 = p.o32 != 0;
 #pragma unroll 1
       for (int c = 0; c < kD / 32; ++c) {
         float a32[32], b32[32];
@@ -716,7 +716,19 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&sm.acc_empty);
         }
-        if (live) {
+        if (live && o32) {
+          // 32-byte stores, each one whole L2 sector of the row (16-byte pieces would leave
+          // every sector half-written by one instruction and cost the L2 a merge)
+#pragma unroll
+          for (int q8 = 0; q8 < 2; ++q8) {
+            uint32_t w[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              w[j] = pack_bf16(fmaf(fp, a32[16 * q8 + 2 * j], fm * b32[16 * q8 + 2 * j]),
+                               fmaf(fp, a32[16 * q8 + 2 * j + 1], fm * b32[16 * q8 + 2 * j + 1]));
+            tc::st_global_32B(orow + c * 32 + q8 * 16, w);
+          }
+        } else if (live) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             float o[8];
@@ -802,6 +814,7 @@ cudaError_t launch_hybrid_commit_tc(const HybridArgs& a, float* S, float* Z, cud
   p.Z = a.Z;
   p.alpha = a.alpha;
   p.O = static_cast<__nv_bfloat16*>(a.O);
+  p.o32 = (reinterpret_cast<uintptr_t>(a.O) & 31) == 0;
   p.dev_err = a.dev_err;
   p.R = a.R;
   p.Hq = a.Hq;

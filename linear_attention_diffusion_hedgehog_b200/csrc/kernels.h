@@ -60,6 +60,7 @@ struct TcHybridParams {
   __nv_bfloat16* O;
   int32_t* dev_err;
   int R, Hq, Hkv, G, T, Bmax, num_slots;  // G = Hq / Hkv query heads per KV head
+  int o32;               // O is 32-byte aligned: rows are written in whole 32-byte sectors
   long long wait_limit;  // SM cycles a bounded wait may spin before giving up
 };
 

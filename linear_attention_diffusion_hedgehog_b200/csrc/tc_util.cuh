@@ -331,6 +331,13 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// 32-byte global store (one whole L2 sector); the address must be 32-byte aligned.
+__device__ __forceinline__ void st_global_32B(void* gptr, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(gptr), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 // Hardware base-2 exponential (MUFU), flush-to-zero; relative error about 2^-22.
 __device__ __forceinline__ float ex2(float x) {
   float y;

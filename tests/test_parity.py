@@ -628,6 +628,58 @@ def test_generic_kernel_extreme_block_logits(sign, prefix):
     assert_close(host64(O), want, dict(rel_l2=1e-4, rel_max=1e-4), "O")
 
 
+def test_decode_step_output_16_byte_aligned_matches_32_byte_aligned():
+    """O rows are written as whole 32-byte sectors when O is 32-byte aligned, and as 16-byte
+    pieces when it is only 16-byte aligned (the alignment the API asks for); the same step
+    into both gives the same bits, for the decode step and for the fused step."""
+    c = inputs.decode_case(R=6, Hq=16, Hkv=4, d=128, F=256, block_lens=[32, 5, 32, 1, 17, 32],
+                           prefix_lens=64, seed=97, dtype="bf16", with_alpha=True)
+    S, Z = build_states_on_gpu(c, block=32)
+    T = int(c.cu_blk[-1])
+    cu = torch.tensor(c.cu_blk, dtype=torch.int32, device="cuda")
+    args = (cu, dev(c.Q, torch.bfloat16), dev(c.K, torch.bfloat16), dev(c.V, torch.bfloat16))
+    W = dev(c.W, torch.bfloat16)
+    alpha = dev(c.alpha, torch.float32)
+    outs = []
+    for shift in (0, 8):  # 8 bf16 = 16 bytes past a 256-byte-aligned allocation
+        buf = torch.full((T * 16 * 128 + 16,), float("nan"), dtype=torch.bfloat16, device="cuda")
+        O = buf[shift:shift + T * 16 * 128].view(T, 16, 128)
+        assert (O.data_ptr() % 32 == 0) == (shift == 0)
+        bha.hybrid_attn(*args, S, Z, W, max_block=32, alpha=alpha, out=O)
+        S2, Z2 = S.clone(), Z.clone()
+        buf2 = torch.full_like(buf, float("nan"))
+        O2 = buf2[shift:shift + T * 16 * 128].view(T, 16, 128)
+        bha.hybrid_attn_commit(*args, S2, Z2, W, max_block=32, alpha=alpha, out=O2)
+        torch.cuda.synchronize()
+        outs.append((O.clone(), O2.clone()))
+    assert torch.equal(outs[0][0], outs[1][0]), "decode step: output depends on O's alignment"
+    assert torch.equal(outs[0][1], outs[1][1]), "fused step: output depends on O's alignment"
+    assert torch.equal(outs[0][0], outs[0][1])
+    So, Zo = oracle_states(c)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, So, Zo, c.W, c.alpha)
+    assert_close(host64(outs[1][0]), want, TOL_BF16, "O (16-byte aligned)")
+
+
+@pytest.mark.parametrize("big_group", [1, 3])
+def test_decode_step_shift_moves_when_a_later_feature_group_dominates(big_group):
+    """The tensor-core step may shift e+ / e- by the max / min of each row's first 32 features
+    and move the shift when a later group passes it.  Here the W columns of one later group
+    are ten times larger, so u there spans about +-30 against +-3 in the first group, and every
+    row's largest and smallest features sit in that group.  States from 64-token prefixes,
+    ragged blocks; every row checked against the oracle."""
+    lens = [32, 7, 32, 1]
+    c = inputs.decode_case(R=4, Hq=16, Hkv=4, d=128, F=256, block_lens=lens, prefix_lens=64,
+                           seed=95 + big_group, dtype="bf16")
+    W = c.W.astype(np.float64).copy()
+    W[:, :, 32 * big_group:32 * big_group + 32] *= 10.0
+    c.W = inputs.bf16_round(W)
+    S, Z = build_states_on_gpu(c, block=32)
+    So, Zo = oracle_states(c)
+    O = run_hybrid(c, S, Z)
+    want = ref.hybrid_attn(c.cu_blk, c.Q, c.K, c.V, So, Zo, c.W)
+    assert_close(host64(O), want, TOL_BF16, "O")
+
+
 # ------------------------------------------------------------------- query heads per KV head
 
 @pytest.mark.parametrize("Hq,Hkv", [(16, 16), (8, 4)])
