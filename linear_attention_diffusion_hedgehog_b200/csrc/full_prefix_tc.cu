@@ -332,16 +332,29 @@ __global__ void __launch_bounds__(kThreads, 1) full_prefix_tc_kernel(const __gri
         if (p.nsplit == 1) {
           const float inv = l > 0.f ? 1.f / l : 0.f;
           __nv_bfloat16* op = p.O + orow * kD;
+          // output rows are not read back here: no L1 allocation, whole 32-byte sectors when
+          // O is 32-byte aligned
+          if (p.o32) {
 #pragma unroll
-          for (int c = 0; c < kD; c += 8)
-            *reinterpret_cast<uint4*>(op + c) =
-                make_uint4(pack_bf16(o[c] * inv, o[c + 1] * inv), pack_bf16(o[c + 2] * inv, o[c + 3] * inv),
-                           pack_bf16(o[c + 4] * inv, o[c + 5] * inv), pack_bf16(o[c + 6] * inv, o[c + 7] * inv));
+            for (int c = 0; c < kD; c += 16) {
+              uint32_t w[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) w[j] = pack_bf16(o[c + 2 * j] * inv, o[c + 2 * j + 1] * inv);
+              tc::st_global_32B(op + c, w);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < kD; c += 8)
+              tc::st_global_16B(op + c, pack_bf16(o[c] * inv, o[c + 1] * inv), pack_bf16(o[c + 2] * inv, o[c + 3] * inv),
+                                pack_bf16(o[c + 4] * inv, o[c + 5] * inv), pack_bf16(o[c + 6] * inv, o[c + 7] * inv));
+          }
         } else {
           const size_t prow = (size_t)x.s * p.T * p.Hq + orow;
           float* op = p.opart + prow * kD;
 #pragma unroll
-          for (int c = 0; c < kD; c += 4) *reinterpret_cast<float4*>(op + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+          for (int c = 0; c < kD; c += 4)
+            tc::st_global_16B(op + c, __float_as_uint(o[c]), __float_as_uint(o[c + 1]), __float_as_uint(o[c + 2]),
+                              __float_as_uint(o[c + 3]));
           p.mpart[prow] = m;
           p.lpart[prow] = l;
         }
@@ -443,6 +456,7 @@ cudaError_t launch_full_prefix_tc(const FullPrefixArgs& a, void* workspace, cuda
   p.cu_blk = a.cu_blk;
   p.kv_len = a.kv_len;
   p.O = static_cast<__nv_bfloat16*>(a.O);
+  p.o32 = (reinterpret_cast<uintptr_t>(a.O) & 31) == 0;
   p.dev_err = a.dev_err;
   p.R = a.R;
   p.Hq = a.Hq;

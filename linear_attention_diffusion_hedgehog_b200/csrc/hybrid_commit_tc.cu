@@ -718,7 +718,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
         }
         if (live && o32) {
           // 32-byte stores, each one whole L2 sector of the row (16-byte pieces would leave
-          // every sector half-written by one instruction and cost the L2 a merge)
+          // every sector half-written by one instruction and cost the L2 a merge), not
+          // allocated in L1
 #pragma unroll
           for (int q8 = 0; q8 < 2; ++q8) {
             uint32_t w[8];
@@ -734,9 +735,8 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_commit_tc_kernel(const __g
             float o[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) o[j] = fmaf(fp, a32[8 * q4 + j], fm * b32[8 * q4 + j]);
-            *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) =
-                make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
-                           pack_bf16(o[6], o[7]));
+            tc::st_global_16B(orow + c * 32 + q4 * 8, pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]),
+                              pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
           }
         }
       }

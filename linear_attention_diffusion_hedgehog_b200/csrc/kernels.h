@@ -95,6 +95,7 @@ struct TcFullParams {
   float* lpart;  // [nsplit][T * Hq] softmax sums
   int32_t* dev_err;
   int R, Hq, Hkv, T, Bmax, cap, nsplit, tiles_per_split;
+  int o32;  // O is 32-byte aligned: rows are written in whole 32-byte sectors
   long long wait_limit;
 };
 

@@ -331,10 +331,17 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       : "memory");
 }
 
-// 32-byte global store (one whole L2 sector); the address must be 32-byte aligned.
+// Global stores of output rows that nothing in the kernel reads back: no L1 allocation.
+// 32-byte form (one whole L2 sector), the address 32-byte aligned.
 __device__ __forceinline__ void st_global_32B(void* gptr, const uint32_t (&w)[8]) {
-  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(gptr), "r"(w[0]),
-               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+  asm volatile("st.global.L1::no_allocate.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(gptr),
+               "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+// 16-byte form, the address 16-byte aligned.
+__device__ __forceinline__ void st_global_16B(void* gptr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.global.L1::no_allocate.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(gptr), "r"(a), "r"(b),
+               "r"(c), "r"(d)
                : "memory");
 }
 
