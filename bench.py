@@ -900,7 +900,8 @@ def bench_per_qhead(args, world, rank, local, steps):
                    UNIT, steps, ms_step, cfg, dtype="bf16", kernel_variant=variant,
                    roofline=_roof(step_bytes(Hkv=HQ), ms_step, peaks, src,
                                   "hybrid tensor-core" if variant == 1 else "hybrid generic",
-                                  flops=step_flops(Hkv=HQ)),
+                                  flops=step_flops(Hkv=HQ),
+                                  traffic=_traffic_for("hybrid_per_qhead", variant, "hybrid_tc.cu")),
                    gpu_launches=steps)
 
 
