@@ -44,8 +44,9 @@
 //               k+1's feature map can start while unit k's P V is still waiting for its P.
 //   warps 2-5   feature map, one warp per TMEM lane quarter and one thread per tile row (its
 //               own TMEM lane): block-softmax max, e+ / e- group by group (each group released
-//               to the MMA as soon as the four warps have written it), P from the scores just
-//               before e- overwrites them, and the epilogue factors for the row.
+//               to the MMA as soon as the four warps have written it), P from the block scores
+//               (saved to registers before e- group 3 overwrites them) once the last group
+//               has gone to the MMA, and the epilogue factors for the row.
 //   warps 6-9   epilogue, one warp per lane quarter: out = f+ A+ + f- A- once the unit's MMAs
 //               are done, each thread storing its row's 16-byte pieces straight from registers
 //               while the feature-map warps already work on the next unit.
@@ -434,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
       const float bpl = mx * log2e + tl2, bml = mn * log2e - tl2;
       const float* zk = sm.z[k & 1];
       float esp = 0.f, esm = 0.f, zsp = 0.f, zsm = 0.f, psum = 0.f;
+      float sv[32];
       bool vgood = true;
 #pragma unroll 1
       for (int c = 0; c < kGroups; ++c) {
@@ -457,37 +459,39 @@ __global__ void __launch_bounds__(kThreads, 1) hybrid_tc_kernel(const __grid_con
           }
           tc::tmem_st16(tl + kColU + c * 32 + 16 * h, ep);
         }
+        // the block scores leave TMEM before e- group 3 overwrites them
         if (c == kGroups - 1) {
-          // sum e+ is complete, so P (bf16, w 2^{s_j} sum e+, or w 2^{s_j - m} for empty
-          // states) is formed now, from the scores that e- group 3 is about to overwrite.  P's
-          // buffer is free once V has landed (V is reloaded only after the previous P V has
-          // completed).
-          vgood = __all_sync(0xffffffffu, tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim));
-          const float lsp = lin ? (esp > 0.f ? tc::lg2(esp) : -tl2) : -m2;
-          float sv[32];
           tc::tmem_ld32(tl + kColS, sv);
           tc::tmem_wait_ld();
-          uint32_t packed[16];
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float a0 = j < x.n ? wgt * tc::ex2(fmaf(sv[j], scale_log2, lsp)) : 0.f;
-            const float a1 = j + 1 < x.n ? wgt * tc::ex2(fmaf(sv[j + 1], scale_log2, lsp)) : 0.f;
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
-            psum += __low2float(b2) + __high2float(b2);
-            packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-          // 64-byte rows, 16-byte chunk c stored at chunk c ^ ((row / 2) % 4) (64-byte swizzle)
-          uint8_t* prow = sm.p + row * 64;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            *reinterpret_cast<uint4*>(prow + ((q4 ^ ((row >> 1) & 3)) << 4)) =
-                make_uint4(packed[4 * q4], packed[4 * q4 + 1], packed[4 * q4 + 2], packed[4 * q4 + 3]);
         }
         tc::tmem_st32(tl + kColEm + c * 32, uu);
         tc::tmem_wait_st();
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&sm.e_ready[c]);
+      }
+      {
+        // sum e+ is complete, so P (bf16, w 2^{s_j} sum e+, or w 2^{s_j - m} for empty
+        // states) is formed now, from the scores saved above, after the last group has gone
+        // to the MMA.  P's buffer is free once V has landed (V is reloaded only after the
+        // previous P V has completed).
+        vgood = __all_sync(0xffffffffu, tc::mbar_wait(&sm.v_full, k & 1, abort_flag, lim));
+        const float lsp = lin ? (esp > 0.f ? tc::lg2(esp) : -tl2) : -m2;
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float a0 = j < x.n ? wgt * tc::ex2(fmaf(sv[j], scale_log2, lsp)) : 0.f;
+          const float a1 = j + 1 < x.n ? wgt * tc::ex2(fmaf(sv[j + 1], scale_log2, lsp)) : 0.f;
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(a0, a1);
+          psum += __low2float(b2) + __high2float(b2);
+          packed[j >> 1] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        // 64-byte rows, 16-byte chunk c stored at chunk c ^ ((row / 2) % 4) (64-byte swizzle)
+        uint8_t* prow = sm.p + row * 64;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+          *reinterpret_cast<uint4*>(prow + ((q4 ^ ((row >> 1) & 3)) << 4)) =
+              make_uint4(packed[4 * q4], packed[4 * q4 + 1], packed[4 * q4 + 2], packed[4 * q4 + 3]);
       }
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&sm.z_empty[k & 1]);
