@@ -48,8 +48,9 @@
 //               (saved to registers before e- group 3 overwrites them) once the last group
 //               has gone to the MMA, and the epilogue factors for the row.
 //   warps 6-9   epilogue, one warp per lane quarter: out = f+ A+ + f- A- once the unit's MMAs
-//               are done, each thread storing its row's 16-byte pieces straight from registers
-//               while the feature-map warps already work on the next unit.
+//               are done, each thread storing its row straight from registers as whole
+//               32-byte sectors, not allocated in L1 (16-byte pieces when O is only 16-byte
+//               aligned), while the feature-map warps already work on the next unit.
 //
 // Every wait is bounded; on expiry the CTA raises BHA_ERR_TIMEOUT in dev_err, drains its
 // own copies and MMAs, frees its TMEM and returns.
