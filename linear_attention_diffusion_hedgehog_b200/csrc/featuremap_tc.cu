@@ -20,10 +20,12 @@
 //               odd ones, matching the TMEM buffers), so one group's exponentials overlap the
 //               other group's read-out and stores.  In a group, warp wq owns TMEM lane quarter
 //               wq and each thread one whole row: max and min of its 128 u values; e+ written
-//               beside u with its sum and read back normalised, 32 rows x 128 bytes at a time,
-//               into a double-buffered staging slot that one asynchronous bulk tensor store
-//               writes to phi; then e- over u in place, likewise.  Storing phi+ before e- is
-//               computed halves the time from a tile's u to its first store.
+//               beside u with its sum and read back normalised, 128 bytes of the row at a
+//               time, each thread storing them as whole 32-byte sectors not allocated in L1
+//               (when phi is only 16-byte aligned: 32 rows x 128 bytes at a time through a
+//               double-buffered staging slot and one asynchronous bulk tensor store); then e-
+//               over u in place, likewise.  Storing phi+ before e- is computed halves the time
+//               from a tile's u to its first store.
 //
 // Every wait is bounded.  On expiry the CTA stops early, the call's output is undefined and
 // BHA_ERR_TIMEOUT goes to dev_err when the caller passed one; nothing traps and TMEM is freed.
@@ -206,6 +208,10 @@ __global__ void __launch_bounds__(kThreads, 1) featuremap_tc_kernel(const __grid
       const int tok_w = t0 + row0 / p.G;       // first token of this warp's rows
       const int head_w = g * p.G + row0 % p.G;  // first head of this warp's rows
       const bool store = tok_w < p.T;
+      // this thread's row of phi: token t0 + row / G, head g G + row % G
+      const int rtok = t0 + (row0 + lane) / p.G, rhead = g * p.G + (row0 + lane) % p.G;
+      const bool rlive = rtok < p.T;
+      char* rowp = static_cast<char*>(p.phi) + ((size_t)rtok * p.H + rhead) * (size_t)(2 * kFh) * (p.out_bf16 ? 2 : 4);
       const int nchunks = p.out_bf16 ? 2 : 4;  // per half
       // normalised read-out of one half (e at TMEM column src), one bulk store per chunk
       auto readout = [&](const int half, const uint32_t src, const float sc, const bool last) {
@@ -237,6 +243,19 @@ __global__ void __launch_bounds__(kThreads, 1) featuremap_tc_kernel(const __grid
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&sm.tm_empty[b]);
           }
+          if (p.o32) {
+            // the row's 128 bytes of this chunk as four whole 32-byte sectors, not in L1
+            if (rlive) {
+              char* dst = rowp + (size_t)f0 * (p.out_bf16 ? 2 : 4);
+#pragma unroll
+              for (int q8 = 0; q8 < 4; ++q8) {
+                uint32_t w[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) w[j] = packed[8 * q8 + j];
+                tc::st_global_32B(dst + q8 * 32, w);
+              }
+            }
+          } else {
           // staging slot nst % 2: its previous store (two stores ago) must have read it
           uint8_t* slot = sm.stg[sw][nst & 1];
           if (lane == 0) bulk_wait_read_one();
@@ -253,6 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) featuremap_tc_kernel(const __grid
               tc::bulk_commit();
             }
             ++nst;
+          }
           }
         }
       };
@@ -339,6 +359,8 @@ cudaError_t launch_featuremap_tc(const void* x, int T, int x_heads, int Hw, cons
   p.Hw = Hw;
   p.G = G;
   p.out_bf16 = out_bf16 ? 1 : 0;
+  p.phi = phi;
+  p.o32 = (reinterpret_cast<uintptr_t>(phi) & 31) == 0;
   p.wait_limit = 2000000000ll;  // about one second of SM cycles
   p.dev_err = dev_err;
 

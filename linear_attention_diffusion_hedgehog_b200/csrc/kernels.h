@@ -102,8 +102,9 @@ struct TcFullParams {
 // Parameters of the tensor-core feature-map kernel (featuremap_tc.cu).
 struct TcFeatParams {
   CUtensorMap tm_x, tm_w, tm_o;
+  void* phi;         // the output, for direct row stores when it is 32-byte aligned
   int32_t* dev_err;  // BHA_ERR_TIMEOUT if a bounded wait gave up; may be null
-  int T, H, Hw, G, out_bf16;
+  int T, H, Hw, G, out_bf16, o32;
   long long wait_limit;
 };
 

@@ -115,6 +115,27 @@ def test_featuremap_tensor_core_head_groupings(H, Hkv, T):
         _check_phi(host64(phi), want, out_dt)
 
 
+def test_featuremap_output_16_byte_aligned_matches_32_byte_aligned():
+    """phi rows are stored as whole 32-byte sectors when the output is 32-byte aligned, and
+    through staged bulk tensor stores when it is only 16-byte aligned (the alignment the API
+    asks for); both give the same bits, fp32 and bf16 output, with a ragged last tile."""
+    rng = np.random.default_rng(77)
+    T, H, Hkv = 301, 16, 4
+    x = dev(inputs.bf16_round(rng.standard_normal((T, H, 128)).astype(np.float32)), torch.bfloat16)
+    W = dev(inputs.bf16_round((rng.standard_normal((Hkv, 128, 128)) / np.sqrt(128)).astype(np.float32)),
+            torch.bfloat16)
+    for out_dt, shift in ((torch.float32, 4), (torch.bfloat16, 8)):  # 16 bytes of the element type
+        outs = []
+        for sh in (0, shift):
+            buf = torch.full((T * H * 256 + shift,), float("nan"), dtype=out_dt, device="cuda")
+            phi = buf[sh:sh + T * H * 256].view(T, H, 256)
+            assert (phi.data_ptr() % 32 == 0) == (sh == 0)
+            bha.featuremap(x, W, out_dtype=out_dt, out=phi)
+            torch.cuda.synchronize()
+            outs.append(phi.clone())
+        assert torch.equal(outs[0], outs[1]), f"{out_dt}: output depends on its alignment"
+
+
 def test_featuremap_group_size_not_a_power_of_two_takes_the_generic_kernel():
     rng = np.random.default_rng(3)
     x = inputs.bf16_round(rng.standard_normal((20, 12, 128)).astype(np.float32))
