@@ -27,7 +27,8 @@
  * - Every call works on the CURRENT CUDA device (cudaGetDevice): its launches, tensor maps and
  *   device limits are those of that device, so all pointers and the stream must belong to it.
  * - All tensor pointers are DEVICE pointers, 16-byte aligned; the caller allocates and owns
- *   every buffer.  The library allocates nothing, keeps no per-call state, never
+ *   every buffer.  Outputs (O, phi) that are also 32-byte aligned are written in whole 32-byte
+ *   sectors, which is faster; the results are the same bits either way.  The library allocates nothing, keeps no per-call state, never
  *   synchronises the stream, and enqueues its kernels on `stream` (a cudaStream_t; NULL is
  *   the legacy default stream).  Calls on different streams touching disjoint buffers may
  *   run concurrently.
