@@ -64,3 +64,17 @@ def test_fused_step_and_commit_bytes():
     R, Hkv, d, F = 128, 4, 128, 256
     assert b.fused_bytes() == b.step_bytes() + R * Hkv * (F * d * 4 + F * 4) == 177_340_416
     assert b.step_bytes() + b.commit_bytes() - b.fused_bytes() == 76_152_832  # S read + Z + K, V, W
+
+
+def test_every_profiled_kernel_has_a_capture_of_its_current_source():
+    """The DRAM traffic each roofline object reports comes from an ncu capture in profiles/
+    whose recorded source hash matches the kernel as it is now; a kernel edited after its
+    capture would report no traffic, so the captures are kept current."""
+    b = _bench()
+    lookups = {"hybrid_decode": "hybrid_tc.cu", "hybrid_per_qhead": "hybrid_tc.cu",
+               "fused": "hybrid_commit_tc.cu", "commit": "commit_tc.cu",
+               "commit_b128": "commit_tc.cu", "featuremap": "featuremap_tc.cu",
+               "teacher_8k": "full_prefix_tc.cu"}
+    for key, src in lookups.items():
+        got = b.profiled_traffic(key, b.source_hash(src))
+        assert got is not None and got > 0, f"{key}: no capture of the current {src}"
